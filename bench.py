@@ -1,0 +1,425 @@
+"""Benchmark of the fine-grained FP8 Linear hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload fprop]
+                    [--impl ours|reference]
+
+A step is one pass of the hot path over one batch of synthetic input on the
+chosen workload (default: the dense-MLP Fprop shape, X[4096,7168] and
+W[18432,7168] in BF16): 1x128 activation quantization, 128x128 weight
+quantization and the block-scaled FP8 GEMM with FP32 promotion per 128-K
+block, BF16 output.  Other workloads (--workload dgrad|wgrad|wgrad_pow2|moe|
+pr1) run the other passes of the Linear the same way.
+
+The metric is FP8 block-scaled GEMM throughput: 2*M*N*K algorithmic FLOPs
+per step divided by the device time of the whole step (quantizers included),
+as TFLOP/s summed over all ranks.  For N > 1 (torchrun) every rank runs an
+independent replica of the workload (weak scaling: the path needs no
+collective); time is the max over ranks.
+
+The JSON line also carries
+  roofline      the GEMM kernel's achieved TFLOP/s (CUDA events around its
+                launches in the timed region) against the FP8 peak derived
+                from the measured BF16 peak x 2 (nominal FP8/BF16 ratio), and
+                the quantizers' GB/s against the measured HBM copy bandwidth;
+  cpu_baseline  the CPU oracle timed on this host on a bounded sample of the
+                same workload (rank 0, N = 1 only), extrapolated to a step;
+  e2e           the same metric through the C ABI with the inputs copied from
+                pinned host memory and the output copied back, every step;
+  clocks        SM clock / throttle reasons sampled with nvidia-smi during the
+                timed region.
+`--impl reference` times the CPU oracle as it stands (the reference arm).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ---------------------------------------------------------------- peaks
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons every 200 ms while active."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- workloads
+
+def make_step(workload, device):
+    import torch
+    from fp8_fine_grained_x1_b200 import SCALE_FP32, SCALE_POW2, linear, synth
+    if workload == "fprop":
+        wl = synth.fprop()
+        step = linear.FpropStep(wl["x"].to(device), wl["w"].to(device))
+        M, K = wl["x"].shape
+        N = wl["w"].shape[0]
+        desc = dict(workload="fprop dense-MLP X[4096,7168] x W[18432,7168]^T, bf16 in, "
+                    "1x128 act / 128x128 weight E4M3, bf16 out", M=M, N=N, K=K)
+        inputs = [wl["x"], wl["w"]]
+        quant_bytes = (M * K + N * K) * 3 + (M * K // 128) * 4 + (N * K // 16384) * 4
+    elif workload == "pr1":
+        wl = synth.pr1()
+        step = linear.FpropStep(wl["x"].to(device), wl["w"].to(device), out_dtype=torch.float32)
+        M, K = wl["x"].shape
+        N = wl["w"].shape[0]
+        desc = dict(workload="pr1 tiny fprop X[128,512] x W[256,512]^T fp32 in, fp32 out",
+                    M=M, N=N, K=K)
+        inputs = [wl["x"], wl["w"]]
+        quant_bytes = (M * K + N * K) * 5
+    elif workload == "dgrad":
+        wl = synth.dgrad()
+        step = linear.DgradStep(wl["dy"].to(device), wl["w"].to(device))
+        M, Kg = wl["dy"].shape
+        N = wl["w"].shape[1]
+        desc = dict(workload="dgrad dX[4096,2048] = dY[4096,7168] . W[7168,2048] (W read "
+                    "transposed), bf16 out", M=M, N=N, K=Kg)
+        K = Kg
+        inputs = [wl["dy"], wl["w"]]
+        quant_bytes = (M * K + K * N) * 3 + (M * K // 128) * 4
+    elif workload in ("wgrad", "wgrad_pow2"):
+        wl = synth.wgrad()
+        mode = SCALE_POW2 if workload == "wgrad_pow2" else SCALE_FP32
+        step = linear.WgradStep(wl["x"].to(device), wl["dy"].to(device), scale_mode=mode)
+        T, C_in = wl["x"].shape
+        C_out = wl["dy"].shape[1]
+        M, N, K = C_out, C_in, T
+        desc = dict(workload=f"wgrad dW[2048,7168] = dY^T . X over 8192 tokens, 128x1 "
+                    f"groups, fp32 out, {'pow2' if mode else 'fp32'} scales", M=M, N=N, K=K)
+        inputs = [wl["x"], wl["dy"]]
+        quant_bytes = (T * C_in + T * C_out) * 3 + (T // 128) * (C_in + C_out) * 4
+    elif workload == "moe":
+        wl = synth.moe()
+        lay = wl["layout"]
+        a = synth.gather_rows(wl["x"].to(device), lay.row_token)
+        step = linear.MoeStep(a, wl["w"].to(device), lay.offsets.to(device))
+        G, N, K = wl["w"].shape
+        M = int(lay.counts.sum())
+        desc = dict(workload="moe grouped fprop, 32 experts W_e[2048,7168], 16384 tokens "
+                    "top-8 Zipf(1.1), groups padded to 128, bf16 out", M=M, N=N, K=K,
+                    M_padded=lay.m_total)
+        inputs = [a.cpu(), wl["w"]]
+        quant_bytes = (lay.m_total * K + G * N * K) * 3 + (lay.m_total * K // 128) * 4
+    else:
+        raise SystemExit(f"unknown workload {workload}")
+    flops = 2 * M * N * K
+    return step, desc, flops, quant_bytes, inputs
+
+
+# ---------------------------------------------------------------- oracle (CPU) timing
+
+def oracle_sample(workload, budget_s: float = 20.0):
+    """Time the CPU oracle on a bounded sample of the workload and extrapolate
+    one step: quantizers timed on a row sample, GEMM on sampled outputs."""
+    import numpy as np
+    import torch
+    import oracle
+    from fp8_fine_grained_x1_b200 import synth
+    oracle.build()
+    if workload != "fprop":
+        workload = "fprop"          # the reference arm is quoted on the default workload
+    M, N, K = 4096, 18432, 7168
+    rows = 64
+    x = synth.activations(rows, K, seed=0, outlier_seed=2)
+    w = synth.normal((256, K), 0.006, 1)
+    xb, wb = synth.bf16_bits(x), synth.bf16_bits(w)
+    t0 = time.perf_counter()
+    qx, sx = oracle.quant_act_1x128(xb)
+    qw, sw = oracle.quant_w_128x128(wb)
+    t_quant = time.perf_counter() - t0
+    quant_elems = rows * K + 256 * K
+    rng = np.random.default_rng(0)
+    npts = 256
+    t_gemm, done = 0.0, 0
+    while t_gemm < budget_s * 0.8 and done < 200000:
+        pts = np.stack([rng.integers(0, rows, npts), rng.integers(0, 256, npts)], 1)
+        t0 = time.perf_counter()
+        oracle.gemm_points(qx, sx, qw, sw, pts)
+        t_gemm += time.perf_counter() - t0
+        done += npts
+        npts = min(npts * 2, 65536)
+    per_point = t_gemm / done
+    per_elem_q = t_quant / quant_elems
+    step_s = per_point * M * N + per_elem_q * (M * K + N * K)
+    flops = 2.0 * M * N * K
+    return dict(value=flops / step_s / 1e12, unit="TFLOP/s", cores=oracle.num_threads(), kind="oracle",
+                sample=f"fprop: 1x128/128x128 quantization of {rows}+256 rows and {done} "
+                       f"GEMM outputs (K=7168, FP64), extrapolated to one 4096x18432x7168 step",
+                step_s=step_s)
+
+
+# ---------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="fprop",
+                    choices=["fprop", "pr1", "dgrad", "wgrad", "wgrad_pow2", "moe"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        t0 = time.perf_counter()
+        res = None
+        for _ in range(max(1, args.warmup)):
+            pass
+        vals = []
+        for _ in range(max(1, args.steps)):
+            res = oracle_sample(args.workload, budget_s=max(2.0, 60.0 / max(1, args.steps)))
+            vals.append(res["value"])
+        total = time.perf_counter() - t0
+        v = sorted(vals)[len(vals) // 2]
+        line = {"impl": "reference", "metric": "FP8 block-scaled GEMM TFLOP/s (step incl. "
+                "quantization)", "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": res["step_s"] * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": "fprop dense-MLP X[4096,7168] x W[18432,7168]^T"},
+                "cpu_baseline": {k: res[k] for k in ("value", "unit", "cores", "kind", "sample")},
+                "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0},
+                "wall_s": total}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import fp8_fine_grained_x1_b200 as fg
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    fg.load_library()
+    assert fg.fp8_device_supported(), "needs an sm_100 GPU"
+
+    step, desc, flops, quant_bytes, host_inputs = make_step(args.workload, device)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = fg.fp8_get_status()
+    if status != fg.FP8_OK:
+        raise SystemExit(f"device status after warm-up: {fg.status_string(status)}")
+
+    # ---- timed region: K steps, GEMM launches bracketed by events
+    ev_q0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_g0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_g1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        time.sleep(0.3)
+        start.record(stream)
+        for i in range(args.steps):
+            ev_q0[i].record(stream)
+            step.quantize()
+            ev_g0[i].record(stream)
+            step.gemm()
+            ev_g1[i].record(stream)
+        stop.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms_total = start.elapsed_time(stop)
+    gemm_ms = sorted(ev_g0[i].elapsed_time(ev_g1[i]) for i in range(args.steps))
+    quant_ms = sorted(ev_q0[i].elapsed_time(ev_g0[i]) for i in range(args.steps))
+    gemm_avg = sum(gemm_ms) / len(gemm_ms)
+    quant_avg = sum(quant_ms) / len(quant_ms)
+    if world > 1:
+        t = torch.tensor([ms_total], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    status = fg.fp8_get_status()
+    if status != fg.FP8_OK:
+        raise SystemExit(f"device status after timing: {fg.status_string(status)}")
+
+    ms_per_step = ms_total / args.steps
+    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    peaks = measured_peaks()
+    fp8_peak = 2.0 * peaks["bf16"]
+    gemm_tflops = flops / (gemm_avg * 1e-3) / 1e12
+    quant_gbs = quant_bytes / (quant_avg * 1e-3) / 1e9
+
+    # ---- end to end through the C ABI: pinned host inputs in, output back
+    e2e = None
+    if args.e2e_steps > 0:
+        pinned = [t.contiguous().pin_memory() for t in host_inputs]
+        dev_inputs = [step_input for step_input in _step_inputs(step)]
+        out_dev = _step_output(step)
+        out_host = torch.empty(out_dev.shape, dtype=out_dev.dtype, pin_memory=True)
+        h2d = sum(t.numel() * t.element_size() for t in pinned)
+        d2h = out_host.numel() * out_host.element_size()
+        for p, d in zip(pinned, dev_inputs):
+            d.copy_(p.view(d.shape), non_blocking=True)
+        step()
+        out_host.copy_(out_dev, non_blocking=True)
+        torch.cuda.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            for p, d in zip(pinned, dev_inputs):
+                d.copy_(p.view(d.shape), non_blocking=True)
+            step()
+            out_host.copy_(out_dev, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1) / args.e2e_steps
+        if world > 1:
+            t = torch.tensor([e_ms], device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res = oracle_sample(args.workload)
+        cpu = {k: res[k] for k in ("value", "unit", "cores", "kind", "sample")}
+
+    if rank == 0:
+        cfg = dict(desc)
+        cfg.update(parallelism=f"replicas x{world}", l2="inputs larger than L2 "
+                   "(no flush)" if sum(t.numel() * t.element_size() for t in host_inputs) > L2_BYTES
+                   else "inputs smaller than L2")
+        line = {
+            "metric": "FP8 block-scaled GEMM TFLOP/s (step incl. quantization)",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 x e4m3 -> f32",
+            "data": "synthetic (seeded torch.Generator draws)", "config": cfg,
+            "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak,
+                         "unit": "TFLOP/s", "frac": gemm_tflops / fp8_peak, "traffic": None,
+                         "kernel": "k_fp8_gemm", "peak_source":
+                         f"{peaks['source']} bf16 burst {peaks['bf16']} x 2 (FP8/BF16 nominal)"},
+            "quantizers": {"achieved_gbs": quant_gbs, "peak_gbs": peaks["hbm"],
+                           "frac": quant_gbs / peaks["hbm"], "ms_per_step": quant_avg,
+                           "algorithmic_bytes": quant_bytes},
+            "gemm_ms": gemm_avg, "gemm_ms_min": gemm_ms[0],
+            "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": step.kernel_calls * args.steps,
+            "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def _step_inputs(step):
+    from fp8_fine_grained_x1_b200 import linear
+    if isinstance(step, linear.FpropStep):
+        return [step.x, step.w]
+    if isinstance(step, linear.DgradStep):
+        return [step.dy, step.w]
+    if isinstance(step, linear.WgradStep):
+        return [step.x, step.dy]
+    return [step.a, step.w]
+
+
+def _step_output(step):
+    from fp8_fine_grained_x1_b200 import linear
+    if isinstance(step, linear.DgradStep):
+        return step.dx
+    if isinstance(step, linear.WgradStep):
+        return step.dw
+    return step.y
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,39 @@
+// fp8fg_host.h -- internal host-side interface between the C ABI (api.cu) and
+// the kernel launchers (quant.cu, gemm.cu).  Arguments reaching these
+// functions have already been validated by api.cu.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace fp8fg {
+
+cudaError_t launch_quant_act_1x128(const void* x, int in_dtype, int64_t M, int64_t K, int64_t ldx,
+                                   uint8_t* q, int64_t ldq, float* sA, int mode, cudaStream_t st);
+cudaError_t launch_quant_act_128x1(const void* x, int in_dtype, int64_t T, int64_t C, int64_t ldx,
+                                   uint8_t* qT, int64_t ldqT, float* s, int mode, cudaStream_t st);
+cudaError_t launch_quant_w_128x128(const void* w, int in_dtype, int64_t N, int64_t K, int64_t ldw,
+                                   uint8_t* q, int64_t ldq, float* sW, int mode, cudaStream_t st);
+
+// Dense (G == 0, group_offsets == nullptr) or grouped block-scaled GEMM.
+// For the grouped form B is [G][N][K] K-major and sB [G][N/128][K/128].
+// Returns cudaSuccess or the launch / tensor-map error; *status_out gets the
+// fp8_status code to report.
+int launch_blockscaled_gemm(const uint8_t* A, const float* sA, const uint8_t* B, int b_major,
+                            const float* sB, int sb_gran, int64_t M, int64_t N, int64_t K,
+                            const int32_t* group_offsets, int G, void* D, int out_dtype,
+                            int64_t ldd, cudaStream_t st);
+
+cudaError_t launch_selftest_wait(cudaStream_t st);
+
+// Synchronise `st`, then read and clear the current device's status word.
+int read_and_clear_status(cudaStream_t st);
+
+// Process-wide settings / device facts.
+uint64_t wait_timeout_ns();
+void set_wait_timeout_ns(uint64_t ns);
+int device_sm_count();          // of the current device (cached per device)
+bool device_is_sm100();         // current device is compute capability 10.x
+
+}  // namespace fp8fg

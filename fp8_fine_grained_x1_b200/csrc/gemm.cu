@@ -1,0 +1,582 @@
+// gemm.cu -- block-scaled E4M3 x E4M3 GEMM with FP32 promotion every 128 K
+// (sm_100a: TMA -> shared memory -> tcgen05.mma.kind::f8f6f4 -> TMEM).
+//
+// What it computes (DeepSeek-V3 FP8 recipe as reproduced on the pages "5 Ways
+// You can get More Deepseek While Spending Less", the why-be.co.kr post and
+// the gnrental.net post, passage on increasing accumulation precision): the
+// scales vary along the inner dimension every 128 elements, so the tensor
+// cores produce one partial product per 128-element K-block, and that partial
+// is moved out, multiplied by scale_a * scale_b and accumulated in full FP32.
+//
+// The pages' H800 design keeps two WGMMA warpgroups in flight so one promotes
+// while the other multiplies.  On sm_100 the same overlap comes from the
+// accumulator living in TMEM: the MMA writes K-block kb's partial into one of
+// two TMEM buffers while the promotion warps drain the other buffer into
+// FP32 registers.  Roles per CTA (persistent, one CTA per SM):
+//   warp 0      TMA producer: A / B tiles for each K-block into a 4-stage
+//               shared-memory ring (128-byte swizzle, no cluster multicast)
+//   warp 1      TMEM allocator + MMA issuer: 4 x tcgen05.mma (K = 32 each)
+//               per K-block into TMEM buffer kb & 1, then tcgen05.commit
+//   warps 2-3   idle (they complete warpgroup 0, which hands its registers
+//               to the promotion warpgroups)
+//   warps 4-11  promotion + epilogue: tcgen05.ld the partial, FMA it (packed
+//               FP32x2) with its scale into a register accumulator, release the
+//               buffer; after the last K-block convert to BF16/FP32 and store.
+// Tile: 128 (M) x 256 (N) x 128 (K); warps 4-7 own columns 0-127, warps 8-11
+// columns 128-255, each warp the 32 TMEM lanes (rows) its id allows.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "fp8fg_device.cuh"
+#include "fp8fg_host.h"
+
+namespace fp8fg {
+
+// The library's status word (one per device; module-scope, not allocated).
+__device__ int g_status = 0;
+
+__device__ void report_error(int code) { atomicCAS(&g_status, 0, code); }
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 128;
+constexpr int NS = 4;                                   // shared-memory stages
+constexpr uint32_t A_BYTES = BM * BK;                   // 16 KB per stage
+constexpr uint32_t B_BYTES = BN * BK;                   // 32 KB per stage
+constexpr int NUM_PROMO_WARPS = 8;
+constexpr int FIRST_PROMO_WARP = 4;                     // warpgroups 1 and 2
+constexpr int NUM_THREADS = 128 + 32 * NUM_PROMO_WARPS; // 384 = 3 warpgroups
+// Register split: launch gives every thread LAUNCH_REGS (65536 / 384 rounded
+// down to 8); warpgroup 0 (TMA, MMA, 2 idle warps) drops to CTRL_REGS and the
+// two promotion warpgroups rise to PROMO_REGS, within the launch total.
+constexpr uint32_t LAUNCH_REGS = 168;
+constexpr uint32_t CTRL_REGS = 40;
+constexpr uint32_t PROMO_REGS = 216;
+static_assert(128 * CTRL_REGS + 256 * PROMO_REGS <= NUM_THREADS * LAUNCH_REGS,
+              "register split exceeds the launch allocation");
+constexpr uint32_t TMEM_COLS = 2 * BN;                  // two FP32 partial buffers
+constexpr int MAX_GROUPS = 1024;
+constexpr int BAND = 16;                                // m-blocks per raster band
+constexpr uint32_t DYN_SMEM = 1024 + NS * (A_BYTES + B_BYTES);
+
+struct GemmParams {
+    const float* sA;               // [K/128][M]
+    const float* sB;               // see fp8_blockscaled_gemm / fp8_grouped_gemm
+    void* D;
+    const int32_t* group_offsets;  // nullptr: dense
+    int64_t M, N, K, ldd;
+    int G;
+    int b_major, sb_gran, out_dtype;
+    int b_box_rows;                // rows of a K-major B box (128 or 256)
+    uint64_t timeout_ns;
+};
+
+// Tile order: bands of BAND m-blocks; inside a band n-blocks outer, m-blocks
+// inner, so the tiles resident at once share a few A row-blocks and B
+// column-blocks in L2.
+__device__ __forceinline__ void tile_coord(int64_t tile, int64_t nmb, int64_t nnb, int64_t& mb,
+                                           int64_t& nb)
+{
+    const int64_t band_tiles = (int64_t)BAND * nnb;
+    const int64_t band = tile / band_tiles;
+    const int64_t r = tile - band * band_tiles;
+    const int64_t mb0 = band * BAND;
+    const int64_t rows = (nmb - mb0 < BAND) ? (nmb - mb0) : BAND;
+    nb = r / rows;
+    mb = mb0 + r % rows;
+}
+
+// Group of the 128-row block starting at row0: the largest e with
+// off[e] <= row0; -1 when row0 >= off[G] (rows outside every group).
+__device__ __forceinline__ int find_group(const int32_t* off, int G, int64_t row0)
+{
+    int lo = 0, hi = G;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if ((int64_t)off[mid] <= row0)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo < G ? lo : -1;
+}
+
+struct Shared {
+    uint64_t full[NS];
+    uint64_t empty[NS];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+    int bad;
+    int32_t off[MAX_GROUPS + 1];
+    float sbw[NUM_PROMO_WARPS][2][128];   // per-warp column scales (sb_gran == 1)
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// ------------------------------------------------------------------ roles
+
+__device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const GemmParams& p,
+                             uint8_t* smem, Shared& sh, int64_t nmb, int64_t nnb, int64_t nkb)
+{
+    volatile int* abort = &sh.abort;
+    int64_t it = 0;   // loads issued so far; stage it % NS, round it / NS
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; ok && tile < nmb * nnb; tile += gridDim.x) {
+        int64_t mb, nb;
+        tile_coord(tile, nmb, nnb, mb, nb);
+        const int64_t m0 = mb * BM, n0 = nb * BN;
+        int g = 0;
+        if (p.group_offsets) {
+            g = find_group(sh.off, p.G, m0);
+            if (g < 0) continue;
+        }
+        const int64_t n_valid = (p.N - n0 < BN) ? (p.N - n0) : BN;
+        const uint32_t b_bytes = (p.b_major == FP8_B_KMAJOR) ? (uint32_t)p.b_box_rows * BK
+                                                             : (uint32_t)n_valid * BK;
+        const int32_t brow = (int32_t)((int64_t)g * p.N + n0);
+        for (int64_t kb = 0; kb < nkb; ++kb) {
+            const int s = (int)(it % NS);
+            const uint32_t ph = (uint32_t)((it / NS) & 1);
+            if (!mbar_wait(&sh.empty[s], ph ^ 1u, abort, p.timeout_ns)) {
+                ok = false;
+                break;
+            }
+            ++it;
+            mbar_arrive_expect_tx(&sh.full[s], A_BYTES + b_bytes);
+            uint8_t* a_dst = smem + s * A_BYTES;
+            uint8_t* b_dst = smem + NS * A_BYTES + s * B_BYTES;
+            tma_load_2d(a_dst, tmA, &sh.full[s], (int32_t)(kb * BK), (int32_t)m0);
+            if (p.b_major == FP8_B_KMAJOR) {
+                tma_load_2d(b_dst, tmB, &sh.full[s], (int32_t)(kb * BK), brow);
+            } else {
+                tma_load_2d(b_dst, tmB, &sh.full[s], (int32_t)n0, (int32_t)(kb * BK));
+                if (n_valid > 128)
+                    tma_load_2d(b_dst + 128 * BK, tmB, &sh.full[s], (int32_t)(n0 + 128),
+                                (int32_t)(kb * BK));
+            }
+        }
+    }
+    // Every copy issued must land before the CTA may exit: stage s received
+    // ceil((it - s) / NS) loads, the last one completing phase (count-1)&1.
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+        const int64_t count = it > s ? (it - s + NS - 1) / NS : 0;
+        if (count) mbar_wait_drain(&sh.full[s], (uint32_t)((count - 1) & 1), p.timeout_ns);
+    }
+}
+
+__device__ void run_mma(const GemmParams& p, uint8_t* smem, Shared& sh, int64_t nmb, int64_t nnb,
+                        int64_t nkb)
+{
+    volatile int* abort = &sh.abort;
+    const uint32_t a_base = smem_u32(smem);
+    const uint32_t b_base = a_base + NS * A_BYTES;
+    const uint32_t tmem = sh.tmem_base;
+    int64_t it = 0, kbg = 0;
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; ok && tile < nmb * nnb; tile += gridDim.x) {
+        int64_t mb, nb;
+        tile_coord(tile, nmb, nnb, mb, nb);
+        const int64_t n0 = nb * BN;
+        if (p.group_offsets && find_group(sh.off, p.G, mb * BM) < 0) continue;
+        const int64_t n_valid = (p.N - n0 < BN) ? (p.N - n0) : BN;
+        const uint32_t idesc = idesc_e4m3_f32(BM, (uint32_t)n_valid, (uint32_t)p.b_major);
+        for (int64_t kb = 0; kb < nkb; ++kb, ++it, ++kbg) {
+            const int s = (int)(it % NS);
+            const uint32_t ph = (uint32_t)((it / NS) & 1);
+            const uint32_t buf = (uint32_t)(kbg & 1);
+            const uint32_t tph = (uint32_t)((kbg >> 1) & 1);
+            if (!mbar_wait(&sh.tempty[buf], tph ^ 1u, abort, p.timeout_ns) ||
+                !mbar_wait(&sh.full[s], ph, abort, p.timeout_ns)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d = tmem + buf * BN;
+            const uint32_t a_addr = a_base + s * A_BYTES;
+            const uint32_t b_addr = b_base + s * B_BYTES;
+#pragma unroll
+            for (int k = 0; k < BK / 32; ++k) {
+                const uint64_t adesc = smem_desc_sw128(a_addr + k * 32, 16, 1024);
+                const uint64_t bdesc = (p.b_major == FP8_B_KMAJOR)
+                                           ? smem_desc_sw128(b_addr + k * 32, 16, 1024)
+                                           : smem_desc_sw128(b_addr + k * 32 * 128, 128 * BK, 1024);
+                mma_f8f6f4(d, adesc, bdesc, idesc, k > 0 ? 1u : 0u);
+            }
+            mma_commit(&sh.empty[s]);     // stage free once these MMAs are done
+            mma_commit(&sh.tfull[buf]);   // partial of this K-block ready
+        }
+    }
+    // Wait for every MMA this thread issued before TMEM is released.
+    mma_commit(&sh.drain);
+    mbar_wait_drain(&sh.drain, 0, p.timeout_ns);
+}
+
+__device__ void run_promotion(const GemmParams& p, Shared& sh, int nmb, int nnb, int nkb, int warp,
+                              int lane)
+{
+    volatile int* abort = &sh.abort;
+    const int ew = warp - FIRST_PROMO_WARP;   // 0..7
+    const int quad = warp & 3;            // TMEM lanes this warp may access
+    const int half = ew >> 2;             // column half of the tile
+    const int row = quad * 32 + lane;     // tile row == TMEM lane
+    const int col0 = half * 128;
+    const uint32_t tmem_lane = sh.tmem_base + ((uint32_t)(quad * 32) << 16);
+    const int nnb128 = (int)(p.N / 128);
+    uint32_t kbg = 0;
+
+    for (int tile = blockIdx.x; tile < nmb * nnb; tile += gridDim.x) {
+        int64_t mb64, nb64;
+        tile_coord(tile, nmb, nnb, mb64, nb64);
+        const int mb = (int)mb64, nb = (int)nb64;
+        const int m0 = mb * BM, n0 = nb * BN;
+        int g = 0;
+        if (p.group_offsets) {
+            g = find_group(sh.off, p.G, m0);
+            if (g < 0) continue;
+        }
+        const int m = m0 + row;
+        const bool row_ok = m < p.M;
+        const bool active = (n0 + col0) < p.N;
+        const int cb = (n0 + col0) / 128;   // 128-column block of B
+
+        // Scales of K-block kb for this thread, prefetched one K-block ahead:
+        //   sa   its row's activation scale, sA[kb][m]
+        //   sb   its 128-column block's weight scale (sb_gran 128), or
+        //   sb4  4 of its half's 128 column scales (sb_gran 1), staged in this
+        //        warp's shared buffer so every lane can read all 128.
+        const float* sa_ptr = p.sA + (row_ok ? m : 0);
+        const int64_t sa_step = row_ok ? p.M : 0;
+        const bool use_sb = active && p.sb_gran == 128;
+        const float* sb_ptr = p.sB;
+        int64_t sb_step = 0;
+        if (p.sb_gran == 128) {
+            if (p.b_major == FP8_B_KMAJOR) {
+                sb_ptr = p.sB + ((int64_t)g * nnb128 + cb) * nkb;
+                sb_step = 1;
+            } else {
+                sb_ptr = p.sB + cb;
+                sb_step = nnb128;
+            }
+        }
+        const bool use_sb4 = active && p.sb_gran == 1;
+        const float4* sb4_ptr = reinterpret_cast<const float4*>(p.sB + n0 + col0) + lane;
+        const int64_t sb4_step = p.N / 4;
+
+        float acc[128];
+#pragma unroll
+        for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+
+        float sa_next = row_ok ? __ldg(sa_ptr) : 0.0f;
+        float sb_next = use_sb ? __ldg(sb_ptr) : 0.0f;
+        if (p.sb_gran == 1) {
+            *reinterpret_cast<float4*>(&sh.sbw[ew][0][lane * 4]) =
+                use_sb4 ? __ldg(sb4_ptr) : make_float4(0.f, 0.f, 0.f, 0.f);
+            __syncwarp();
+        }
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb, ++kbg) {
+            const float sa = sa_next, sb = sb_next;
+            float4 sb4_next = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (kb + 1 < nkb) {
+                sa_ptr += sa_step;
+                sb_ptr += sb_step;
+                sb4_ptr += sb4_step;
+                if (row_ok) sa_next = __ldg(sa_ptr);
+                if (use_sb) sb_next = __ldg(sb_ptr);
+                if (use_sb4) sb4_next = __ldg(sb4_ptr);
+            }
+            const uint32_t buf = kbg & 1;
+            const uint32_t tph = (kbg >> 1) & 1;
+            if (!mbar_wait(&sh.tfull[buf], tph, abort, p.timeout_ns)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            if (active) {
+                const uint32_t taddr = tmem_lane + buf * BN + col0;
+                if (p.sb_gran == 128) {
+                    const float sc = sa * sb;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        uint32_t r[16];
+                        tmem_ld16(taddr + c * 16, r);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            ffma2(acc[c * 16 + 2 * i], acc[c * 16 + 2 * i + 1],
+                                  __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), sc, sc);
+                    }
+                } else {
+                    const float* sbv = sh.sbw[ew][kb & 1];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        uint32_t r[16];
+                        tmem_ld16(taddr + c * 16, r);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float4 b = *reinterpret_cast<const float4*>(sbv + c * 16 + 4 * i);
+                            float t0, t1, t2, t3;
+                            fmul2(t0, t1, b.x, b.y, sa, sa);
+                            fmul2(t2, t3, b.z, b.w, sa, sa);
+                            const int j = c * 16 + 4 * i;
+                            ffma2(acc[j], acc[j + 1], __uint_as_float(r[4 * i]),
+                                  __uint_as_float(r[4 * i + 1]), t0, t1);
+                            ffma2(acc[j + 2], acc[j + 3], __uint_as_float(r[4 * i + 2]),
+                                  __uint_as_float(r[4 * i + 3]), t2, t3);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.tempty[buf]);
+            if (p.sb_gran == 1) {
+                *reinterpret_cast<float4*>(&sh.sbw[ew][(kb + 1) & 1][lane * 4]) = sb4_next;
+                __syncwarp();
+            }
+        }
+        if (!ok) break;
+
+        // Epilogue: round the FP32 sums to the output type and store the row.
+        if (active && row_ok) {
+            if (p.out_dtype == FP8_OUT_BF16) {
+                __nv_bfloat16* drow =
+                    static_cast<__nv_bfloat16*>(p.D) + (int64_t)m * p.ldd + n0 + col0;
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    uint4 v;
+                    v.x = pack_bf16x2(acc[8 * c + 0], acc[8 * c + 1]);
+                    v.y = pack_bf16x2(acc[8 * c + 2], acc[8 * c + 3]);
+                    v.z = pack_bf16x2(acc[8 * c + 4], acc[8 * c + 5]);
+                    v.w = pack_bf16x2(acc[8 * c + 6], acc[8 * c + 7]);
+                    *reinterpret_cast<uint4*>(drow + 8 * c) = v;
+                }
+            } else {
+                float* drow = static_cast<float*>(p.D) + (int64_t)m * p.ldd + n0 + col0;
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                    *reinterpret_cast<float4*>(drow + 4 * c) =
+                        make_float4(acc[4 * c], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]);
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    k_fp8_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const GemmParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ Shared sh;
+    // Operand tiles need 1024-byte alignment (128-byte swizzle atoms).
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t nmb = (p.M + BM - 1) / BM;
+    const int64_t nnb = (p.N + BN - 1) / BN;
+    const int64_t nkb = p.K / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&sh.full[s], 1);
+            mbar_init(&sh.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sh.tfull[b], 1);
+            mbar_init(&sh.tempty[b], NUM_PROMO_WARPS);
+        }
+        mbar_init(&sh.drain, 1);
+        sh.abort = 0;
+        sh.bad = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(&sh.tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (p.group_offsets)
+        for (int i = threadIdx.x; i <= p.G; i += NUM_THREADS) sh.off[i] = p.group_offsets[i];
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (p.group_offsets && threadIdx.x == 0) {
+        bool bad = sh.off[0] != 0 || (int64_t)sh.off[p.G] > p.M;
+        for (int e = 0; e < p.G; ++e) bad = bad || sh.off[e + 1] < sh.off[e] || (sh.off[e + 1] & 127);
+        if (bad) {
+            sh.bad = 1;
+            if (blockIdx.x == 0) report_error(FP8_ERR_SHAPE);
+        }
+    }
+    __syncthreads();
+
+    if (warp < FIRST_PROMO_WARP) {
+        regs_dec<CTRL_REGS>();
+        if (!sh.bad) {
+            if (warp == 0) {
+                if (lane == 0) run_producer(&tmA, &tmB, p, smem, sh, nmb, nnb, nkb);
+                __syncwarp();
+            } else if (warp == 1) {
+                if (lane == 0) run_mma(p, smem, sh, nmb, nnb, nkb);
+                __syncwarp();
+            }
+        }
+    } else {
+        regs_inc<PROMO_REGS>();
+        if (!sh.bad) run_promotion(p, sh, (int)nmb, (int)nnb, (int)nkb, warp, lane);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(sh.tmem_base, TMEM_COLS);
+}
+
+__global__ void k_selftest_wait(uint64_t timeout_ns)
+{
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    // Nothing ever arrives on `bar`: the wait runs into its time limit.
+    if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, timeout_ns);
+}
+
+// ------------------------------------------------------------------ host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+// 2-D uint8 tensor [outer][inner] with rows `row_bytes` apart; boxes of
+// box_inner x box_outer bytes, 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool ensure_smem_attr()
+{
+    // once per device
+    static bool done[64] = {};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!done[dev]) {
+        if (cudaFuncSetAttribute(k_fp8_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)DYN_SMEM) != cudaSuccess)
+            return false;
+        done[dev] = true;
+    }
+    return true;
+}
+
+}  // namespace
+
+int launch_blockscaled_gemm(const uint8_t* A, const float* sA, const uint8_t* B, int b_major,
+                            const float* sB, int sb_gran, int64_t M, int64_t N, int64_t K,
+                            const int32_t* group_offsets, int G, void* D, int out_dtype,
+                            int64_t ldd, cudaStream_t st)
+{
+    if (M == 0) return FP8_OK;
+    CUtensorMap tmA, tmB;
+    const int b_box_rows = N >= BN ? BN : (int)N;
+    if (!make_map(&tmA, A, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, BM)) return FP8_ERR_LAUNCH;
+    bool okB;
+    if (b_major == FP8_B_KMAJOR) {
+        const uint64_t rows = (uint64_t)N * (uint64_t)(group_offsets ? G : 1);
+        okB = make_map(&tmB, B, (uint64_t)K, rows, (uint64_t)K, BK, (uint32_t)b_box_rows);
+    } else {
+        okB = make_map(&tmB, B, (uint64_t)N, (uint64_t)K, (uint64_t)N, 128, BK);
+    }
+    if (!okB) return FP8_ERR_LAUNCH;
+    if (!ensure_smem_attr()) return FP8_ERR_LAUNCH;
+
+    GemmParams p;
+    p.sA = sA;
+    p.sB = sB;
+    p.D = D;
+    p.group_offsets = group_offsets;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.ldd = ldd;
+    p.G = group_offsets ? G : 0;
+    p.b_major = b_major;
+    p.sb_gran = sb_gran;
+    p.out_dtype = out_dtype;
+    p.b_box_rows = b_box_rows;
+    p.timeout_ns = wait_timeout_ns();
+
+    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int sms = device_sm_count();
+    const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
+    k_fp8_gemm<<<grid, NUM_THREADS, DYN_SMEM, st>>>(tmA, tmB, p);
+    return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_LAUNCH;
+}
+
+cudaError_t launch_selftest_wait(cudaStream_t st)
+{
+    k_selftest_wait<<<1, 32, 0, st>>>(wait_timeout_ns());
+    return cudaGetLastError();
+}
+
+// Synchronise, then read and clear the status word of the current device.
+int read_and_clear_status(cudaStream_t st)
+{
+    if (cudaStreamSynchronize(st) != cudaSuccess) return FP8_ERR_DEVICE;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return FP8_ERR_DEVICE;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return FP8_ERR_DEVICE;
+    return v;
+}
+
+}  // namespace fp8fg

@@ -1,0 +1,351 @@
+// quant.cu -- online E4M3 quantizers of the fine-grained FP8 Linear (sm_100a).
+//
+// Three HBM-bound kernels, one per grouping of the DeepSeek-V3 FP8 recipe
+// (pages: why-be.co.kr post, cameseeing.com post and "Three Fast Methods To
+// Study Deepseek", Figure 7 (a); "5 Ways You can get More Deepseek While
+// Spending Less", max-abs -> FP8 maximum and power-of-2 scales):
+//   k_quant_1x128    one scale per token per 128 channels
+//   k_quant_128x1    one scale per channel per 128 tokens, written transposed
+//   k_quant_w128     one scale per 128x128 weight block
+// Each reads its input once with 16-byte vector loads, reduces the group's
+// max-abs with warp shuffles (plus shared memory for the wider groups),
+// derives the scale with correctly rounded FP32 division, and writes packed
+// E4M3 codes (cvt.rn.satfinite.e4m3x2) with 8- or 16-byte stores.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "fp8fg_device.cuh"
+#include "fp8fg_host.h"
+
+namespace fp8fg {
+
+namespace {
+
+// ------------------------------------------------------------ group scale
+
+struct GroupScale {
+    float s;    // stored scale (dequantisation multiplier)
+    float inv;  // factor applied before the E4M3 cast
+};
+
+// Scale of a group with max-abs `amax` (amax >= 0, finite).
+//   FP32 mode: s = amax/448, inv = 448/amax, both correctly rounded; a zero
+//              group gets s = inv = 1; when amax/448 would fall below the
+//              smallest normal FP32 the scale saturates at 2^-126.
+//   POW2 mode: s = 2^e, e least with amax <= 448*2^e, e >= -126; inv = 2^-e.
+__device__ __forceinline__ GroupScale group_scale(float amax, int mode)
+{
+    GroupScale g;
+    if (amax == 0.0f) {
+        g.s = 1.0f;
+        g.inv = 1.0f;
+        return g;
+    }
+    if (mode == FP8_SCALE_POW2) {
+        const uint32_t b = __float_as_uint(amax);
+        const int ex = (int)((b >> 23) & 0xFF);
+        int e = -126;
+        if (ex != 0) {
+            // amax = m * 2^(ex-127), m in [1,2).  448 = 1.75 * 2^8, so the
+            // least e is ex-127-8 when m <= 1.75 and one more otherwise.
+            e = ex - 127 - 8 + (((b & 0x7FFFFFu) > 0x600000u) ? 1 : 0);
+            if (e < -126) e = -126;
+        }
+        g.s = __uint_as_float((uint32_t)(e + 127) << 23);
+        g.inv = __uint_as_float((uint32_t)(127 - e) << 23);
+        return g;
+    }
+    if (amax < __uint_as_float(0x04E00000u)) {        // 1.75 * 2^-118
+        g.s = __uint_as_float(0x00800000u);            // 2^-126
+        g.inv = __uint_as_float(0x7E800000u);          // 2^126
+        return g;
+    }
+    g.inv = __fdiv_rn(448.0f, amax);
+    g.s = __fdiv_rn(amax, 448.0f);
+    return g;
+}
+
+// Four scaled values -> four E4M3 codes packed little-endian in a uint32.
+__device__ __forceinline__ uint32_t encode4(float a, float b, float c, float d, float inv)
+{
+    const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fmul_rn(a, inv), __fmul_rn(b, inv)), __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fmul_rn(c, inv), __fmul_rn(d, inv)), __NV_SATFINITE, __NV_E4M3);
+    return (uint32_t)lo | ((uint32_t)hi << 16);
+}
+
+// ------------------------------------------------------------ vector loads
+
+__device__ __forceinline__ uint4 ld_stream16(const void* p)
+{
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Eight consecutive input elements held as raw bits (16 B of BF16 or 32 B of
+// FP32) until they are needed as floats.
+template <typename Tin>
+struct Chunk8;
+
+template <>
+struct Chunk8<__nv_bfloat16> {
+    uint4 r;
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) { r = ld_stream16(p); }
+    __device__ __forceinline__ void zero() { r = make_uint4(0, 0, 0, 0); }
+    __device__ __forceinline__ void get(float (&v)[8]) const
+    {
+        v[0] = bf16_lo(r.x); v[1] = bf16_hi(r.x); v[2] = bf16_lo(r.y); v[3] = bf16_hi(r.y);
+        v[4] = bf16_lo(r.z); v[5] = bf16_hi(r.z); v[6] = bf16_lo(r.w); v[7] = bf16_hi(r.w);
+    }
+};
+
+template <>
+struct Chunk8<float> {
+    uint4 a, b;
+    __device__ __forceinline__ void load(const float* p)
+    {
+        a = ld_stream16(p);
+        b = ld_stream16(p + 4);
+    }
+    __device__ __forceinline__ void zero() { a = b = make_uint4(0, 0, 0, 0); }
+    __device__ __forceinline__ void get(float (&v)[8]) const
+    {
+        v[0] = __uint_as_float(a.x); v[1] = __uint_as_float(a.y);
+        v[2] = __uint_as_float(a.z); v[3] = __uint_as_float(a.w);
+        v[4] = __uint_as_float(b.x); v[5] = __uint_as_float(b.y);
+        v[6] = __uint_as_float(b.z); v[7] = __uint_as_float(b.w);
+    }
+};
+
+__device__ __forceinline__ float absmax8(const float (&v)[8])
+{
+    float a = fabsf(v[0]);
+#pragma unroll
+    for (int i = 1; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
+    return a;
+}
+
+// ------------------------------------------------------------ 1x128
+
+constexpr int kRowsPerCta1x128 = 64;   // 16 groups in flight x 4 per thread
+
+// CTA = 256 threads = 16 half-warps; a half-warp owns one 1x128 group at a
+// time (16 lanes x 8 elements); each thread keeps 4 groups' loads in flight.
+// Grid: x = ceil(M/64) row blocks, y = K/128 K-blocks.
+template <typename Tin>
+__global__ void __launch_bounds__(256) k_quant_1x128(const Tin* __restrict__ x, int64_t M,
+                                                     int64_t ldx, uint8_t* __restrict__ q,
+                                                     int64_t ldq, float* __restrict__ sA, int mode)
+{
+    const int h = threadIdx.x >> 4;
+    const int l = threadIdx.x & 15;
+    const int64_t kb = blockIdx.y;
+    const int64_t m0 = (int64_t)blockIdx.x * kRowsPerCta1x128;
+
+    Chunk8<Tin> c[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int64_t m = m0 + u * 16 + h;
+        if (m < M)
+            c[u].load(x + m * ldx + kb * 128 + l * 8);
+        else
+            c[u].zero();
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int64_t m = m0 + u * 16 + h;
+        float v[8];
+        c[u].get(v);
+        float a = absmax8(v);
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 8));
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+        const GroupScale g = group_scale(a, mode);
+        if (m < M) {
+            uint2 out;
+            out.x = encode4(v[0], v[1], v[2], v[3], g.inv);
+            out.y = encode4(v[4], v[5], v[6], v[7], g.inv);
+            *reinterpret_cast<uint2*>(q + m * ldq + kb * 128 + l * 8) = out;
+            if (l == 0) sA[kb * M + m] = g.s;
+        }
+    }
+}
+
+// ------------------------------------------------------------ 128x128
+
+// CTA = 256 threads per 128x128 block: thread (r0 = tid/16, c = tid%16) loads
+// rows r0 + 16 i (i < 8), elements c*8 .. c*8+7 of the block's row segment.
+// Grid: x = K/128, y = N/128.
+template <typename Tin>
+__global__ void __launch_bounds__(256) k_quant_w128(const Tin* __restrict__ w, int64_t ldw,
+                                                    uint8_t* __restrict__ q, int64_t ldq,
+                                                    float* __restrict__ sW, int64_t nkb, int mode)
+{
+    __shared__ float red[8];
+    const int c = threadIdx.x & 15;
+    const int r0 = threadIdx.x >> 4;
+    const int64_t kb = blockIdx.x;
+    const int64_t nb = blockIdx.y;
+    const Tin* base = w + (nb * 128 + r0) * ldw + kb * 128 + c * 8;
+
+    Chunk8<Tin> ch[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ch[i].load(base + (int64_t)(16 * i) * ldw);
+
+    float a = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        float v[8];
+        ch[i].get(v);
+        a = fmaxf(a, absmax8(v));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+    __syncthreads();
+    a = red[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) a = fmaxf(a, red[i]);
+    const GroupScale g = group_scale(a, mode);
+
+    uint8_t* qb = q + (nb * 128 + r0) * ldq + kb * 128 + c * 8;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        float v[8];
+        ch[i].get(v);
+        uint2 out;
+        out.x = encode4(v[0], v[1], v[2], v[3], g.inv);
+        out.y = encode4(v[4], v[5], v[6], v[7], g.inv);
+        *reinterpret_cast<uint2*>(qb + (int64_t)(16 * i) * ldq) = out;
+    }
+    if (threadIdx.x == 0) sW[nb * nkb + kb] = g.s;
+}
+
+// ------------------------------------------------------------ 128x1
+
+constexpr int kTok = 128;   // tokens per tile (one group along tokens)
+constexpr int kCh = 64;     // channels per tile
+
+// CTA = 256 threads per tile of 128 tokens x 64 channels.  The tile is staged
+// in shared memory with coalesced 16-byte row loads; then thread
+// (c = tid%64, quarter = tid/64) walks 32 tokens of channel c, the four
+// quarters combine their max-abs, and each thread writes its 32 codes as two
+// 16-byte stores into the transposed output row qT[c].
+// Grid: x = ceil(C/64), y = T/128.
+template <typename Tin>
+__global__ void __launch_bounds__(256) k_quant_128x1(const Tin* __restrict__ x, int64_t C,
+                                                     int64_t ldx, uint8_t* __restrict__ qT,
+                                                     int64_t ldqT, float* __restrict__ s, int mode)
+{
+    constexpr int kElemsPerChunk = 16 / (int)sizeof(Tin);
+    constexpr int kChunksPerRow = kCh / kElemsPerChunk;
+    constexpr int kChunksPerThread = kTok * kChunksPerRow / 256;
+    __shared__ __align__(16) Tin tile[kTok][kCh];
+    __shared__ float part[4][kCh];
+
+    const int64_t tb = blockIdx.y;
+    const int64_t c0 = (int64_t)blockIdx.x * kCh;
+
+    // 1. stage the tile (channels beyond C are zero; C % 8 == 0)
+    uint4 buf[kChunksPerThread];
+#pragma unroll
+    for (int i = 0; i < kChunksPerThread; ++i) {
+        const int id = threadIdx.x + 256 * i;
+        const int r = id / kChunksPerRow;
+        const int j = id % kChunksPerRow;
+        const int64_t ch = c0 + j * kElemsPerChunk;
+        buf[i] = (ch < C) ? ld_stream16(x + (tb * kTok + r) * ldx + ch) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < kChunksPerThread; ++i) {
+        const int id = threadIdx.x + 256 * i;
+        const int r = id / kChunksPerRow;
+        const int j = id % kChunksPerRow;
+        *reinterpret_cast<uint4*>(&tile[r][j * kElemsPerChunk]) = buf[i];
+    }
+    __syncthreads();
+
+    // 2. column max-abs over 4 x 32 tokens
+    const int c = threadIdx.x % kCh;
+    const int qtr = threadIdx.x / kCh;
+    float v[32];
+    float a = 0.0f;
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+        v[t] = (float)tile[qtr * 32 + t][c];
+        a = fmaxf(a, fabsf(v[t]));
+    }
+    part[qtr][c] = a;
+    __syncthreads();
+    a = fmaxf(fmaxf(part[0][c], part[1][c]), fmaxf(part[2][c], part[3][c]));
+    const GroupScale g = group_scale(a, mode);
+
+    // 3. encode 32 tokens of channel c, store transposed
+    const int64_t ch = c0 + c;
+    if (ch < C) {
+        uint32_t w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            w[i] = encode4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3], g.inv);
+        uint4* dst = reinterpret_cast<uint4*>(qT + ch * ldqT + tb * kTok + qtr * 32);
+        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        if (qtr == 0) s[tb * C + ch] = g.s;
+    }
+}
+
+}  // namespace
+
+// ------------------------------------------------------------ launchers
+
+cudaError_t launch_quant_act_1x128(const void* x, int in_dtype, int64_t M, int64_t K, int64_t ldx,
+                                   uint8_t* q, int64_t ldq, float* sA, int mode, cudaStream_t st)
+{
+    const dim3 grid((unsigned)((M + kRowsPerCta1x128 - 1) / kRowsPerCta1x128), (unsigned)(K / 128));
+    if (in_dtype == FP8_IN_BF16)
+        k_quant_1x128<__nv_bfloat16><<<grid, 256, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(x), M, ldx, q, ldq, sA, mode);
+    else
+        k_quant_1x128<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), M, ldx, q, ldq,
+                                                   sA, mode);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_act_128x1(const void* x, int in_dtype, int64_t T, int64_t C, int64_t ldx,
+                                   uint8_t* qT, int64_t ldqT, float* s, int mode, cudaStream_t st)
+{
+    const dim3 grid((unsigned)((C + kCh - 1) / kCh), (unsigned)(T / kTok));
+    if (in_dtype == FP8_IN_BF16)
+        k_quant_128x1<__nv_bfloat16><<<grid, 256, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(x), C, ldx, qT, ldqT, s, mode);
+    else
+        k_quant_128x1<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), C, ldx, qT,
+                                                   ldqT, s, mode);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_w_128x128(const void* w, int in_dtype, int64_t N, int64_t K, int64_t ldw,
+                                   uint8_t* q, int64_t ldq, float* sW, int mode, cudaStream_t st)
+{
+    const dim3 grid((unsigned)(K / 128), (unsigned)(N / 128));
+    if (in_dtype == FP8_IN_BF16)
+        k_quant_w128<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w),
+                                                          ldw, q, ldq, sW, K / 128, mode);
+    else
+        k_quant_w128<float><<<grid, 256, 0, st>>>(static_cast<const float*>(w), ldw, q, ldq, sW,
+                                                  K / 128, mode);
+    return cudaGetLastError();
+}
+
+}  // namespace fp8fg

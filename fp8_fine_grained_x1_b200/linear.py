@@ -1,0 +1,148 @@
+"""The fine-grained FP8 Linear's three GEMM passes and the MoE expert pass, as
+ready-to-run steps over device-resident inputs.
+
+Each step owns its output buffers (allocated once with torch) and, when
+called, issues only library calls on the current stream:
+
+  FpropStep    X[M,K] --1x128--> (qX, sX);  W[N,K] --128x128--> (qW, sW);
+               Y[M,N] = qX . qW^T                      (BF16 or FP32 out)
+  DgradStep    dY[M,N_out] --1x128--> ;  W[N_out,K_in] --128x128--> (stored
+               orientation); dX[M,K_in] = dY . W, W read MN-major
+  WgradStep    X[T,C_in], dY[T,C_out] --128x1--> token-contiguous codes with
+               per-channel scales; dW[C_out,C_in] = dY^T . X, FP32 out
+  MoeStep      expert-ordered rows A[M_total,K] --1x128-->; W[G,N,K]
+               --128x128-->; grouped GEMM per expert
+
+("5 Ways You can get More Deepseek While Spending Less", Figure 6: Fprop,
+Dgrad and Wgrad all run in FP8; why-be.co.kr / cameseeing.com posts and
+"Three Fast Methods To Study Deepseek", Figure 7 (a): 1x128 / 128x128
+grouping; gnrental.net post: BF16 or FP32 GEMM outputs.)
+
+`kernel_calls` on each step counts the kernels one call launches.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (B_KMAJOR, B_MNMAJOR, SCALE_FP32, fp8_blockscaled_gemm, fp8_grouped_gemm,
+               fp8_quant_act_128x1, fp8_quant_act_1x128, fp8_quant_w_128x128)
+
+
+def _empty(shape, dtype, device):
+    return torch.empty(shape, dtype=dtype, device=device)
+
+
+class FpropStep:
+    kernel_calls = 3
+
+    def __init__(self, x, w, out_dtype=torch.bfloat16, scale_mode=SCALE_FP32):
+        M, K = x.shape
+        N = w.shape[0]
+        d = x.device
+        self.x, self.w, self.mode = x, w, scale_mode
+        self.qx, self.sx = _empty((M, K), torch.uint8, d), _empty((K // 128, M), torch.float32, d)
+        self.qw, self.sw = _empty((N, K), torch.uint8, d), _empty((N // 128, K // 128), torch.float32, d)
+        self.y = _empty((M, N), out_dtype, d)
+        self.flops = 2 * M * N * K
+
+    def quantize(self, stream=None):
+        fp8_quant_act_1x128(self.x, self.qx, self.sx, self.mode, stream)
+        fp8_quant_w_128x128(self.w, self.qw, self.sw, self.mode, stream)
+
+    def gemm(self, stream=None):
+        fp8_blockscaled_gemm(self.qx, self.sx, self.qw, self.sw, self.y, B_KMAJOR, 128, stream)
+
+    def __call__(self, stream=None):
+        self.quantize(stream)
+        self.gemm(stream)
+        return self.y
+
+
+class DgradStep:
+    kernel_calls = 3
+
+    def __init__(self, dy, w, out_dtype=torch.bfloat16, scale_mode=SCALE_FP32):
+        M, N_out = dy.shape
+        N_out2, K_in = w.shape
+        assert N_out == N_out2
+        d = dy.device
+        self.dy, self.w, self.mode = dy, w, scale_mode
+        self.qdy = _empty((M, N_out), torch.uint8, d)
+        self.sdy = _empty((N_out // 128, M), torch.float32, d)
+        self.qw = _empty((N_out, K_in), torch.uint8, d)
+        self.sw = _empty((N_out // 128, K_in // 128), torch.float32, d)
+        self.dx = _empty((M, K_in), out_dtype, d)
+        self.flops = 2 * M * K_in * N_out
+
+    def quantize(self, stream=None):
+        fp8_quant_act_1x128(self.dy, self.qdy, self.sdy, self.mode, stream)
+        fp8_quant_w_128x128(self.w, self.qw, self.sw, self.mode, stream)
+
+    def gemm(self, stream=None):
+        # B = W stored [K = N_out][N = K_in]: MN-major; its block scales
+        # sW[N_out/128][K_in/128] are [K/128][N/128] in GEMM terms.
+        fp8_blockscaled_gemm(self.qdy, self.sdy, self.qw, self.sw, self.dx, B_MNMAJOR, 128, stream)
+
+    def __call__(self, stream=None):
+        self.quantize(stream)
+        self.gemm(stream)
+        return self.dx
+
+
+class WgradStep:
+    kernel_calls = 3
+
+    def __init__(self, x, dy, scale_mode=SCALE_FP32):
+        T, C_in = x.shape
+        T2, C_out = dy.shape
+        assert T == T2
+        d = x.device
+        self.x, self.dy, self.mode = x, dy, scale_mode
+        self.qxT = _empty((C_in, T), torch.uint8, d)
+        self.sx = _empty((T // 128, C_in), torch.float32, d)
+        self.qdyT = _empty((C_out, T), torch.uint8, d)
+        self.sdy = _empty((T // 128, C_out), torch.float32, d)
+        self.dw = _empty((C_out, C_in), torch.float32, d)
+        self.flops = 2 * C_out * C_in * T
+
+    def quantize(self, stream=None):
+        fp8_quant_act_128x1(self.dy, self.qdyT, self.sdy, self.mode, stream)
+        fp8_quant_act_128x1(self.x, self.qxT, self.sx, self.mode, stream)
+
+    def gemm(self, stream=None):
+        fp8_blockscaled_gemm(self.qdyT, self.sdy, self.qxT, self.sx, self.dw, B_KMAJOR, 1, stream)
+
+    def __call__(self, stream=None):
+        self.quantize(stream)
+        self.gemm(stream)
+        return self.dw
+
+
+class MoeStep:
+    kernel_calls = 3
+
+    def __init__(self, a, w, offsets, out_dtype=torch.bfloat16, scale_mode=SCALE_FP32):
+        M_total, K = a.shape
+        G, N, K2 = w.shape
+        assert K == K2
+        d = a.device
+        self.a, self.w, self.offsets, self.mode = a, w, offsets, scale_mode
+        self.qa = _empty((M_total, K), torch.uint8, d)
+        self.sa = _empty((K // 128, M_total), torch.float32, d)
+        self.qw = _empty((G, N, K), torch.uint8, d)
+        self.sw = _empty((G, N // 128, K // 128), torch.float32, d)
+        self.y = _empty((M_total, N), out_dtype, d)
+
+    def quantize(self, stream=None):
+        fp8_quant_act_1x128(self.a, self.qa, self.sa, self.mode, stream)
+        G, N, K = self.w.shape
+        fp8_quant_w_128x128(self.w.view(G * N, K), self.qw.view(G * N, K),
+                            self.sw.view(G * N // 128, K // 128), self.mode, stream)
+
+    def gemm(self, stream=None):
+        fp8_grouped_gemm(self.qa, self.sa, self.qw, self.sw, self.offsets, self.y, stream)
+
+    def __call__(self, stream=None):
+        self.quantize(stream)
+        self.gemm(stream)
+        return self.y

@@ -159,3 +159,22 @@ def moe(tokens: int = 16384, experts: int = 32, k: int = 8, N: int = EXPERT_HIDD
     layout = moe_layout(zipf_topk_routing(tokens, experts, k, seed=3), experts)
     w = normal((experts, N, K), 0.006, 1)
     return dict(x=x, w=w, layout=layout)
+
+
+# --------------------------------------------------------------------------
+# Raw operands for GEMM-only cases
+# --------------------------------------------------------------------------
+
+def random_e4m3_codes(shape, seed: int):
+    """Uniformly drawn finite E4M3FN byte codes (every byte except 0x7F, 0xFF)."""
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    finite = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    return finite[rng.integers(0, len(finite), shape)]
+
+
+def random_scales(shape, seed: int, lo: float = -12.0, hi: float = 4.0):
+    """FP32 values 2^u with u ~ U(lo, hi)."""
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    return np.exp2(rng.uniform(lo, hi, shape)).astype(np.float32)

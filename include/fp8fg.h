@@ -1,0 +1,206 @@
+/*
+ * fp8fg.h -- C ABI of libfp8fg: the fine-grained FP8 Linear operator on B200
+ * (sm_100a).  Online E4M3 quantization (1x128 activation tiles, 128x1
+ * token-axis tiles for Wgrad, 128x128 weight blocks) and the block-scaled
+ * E4M3 x E4M3 GEMM with FP32 promotion of every 128-element K partial, for
+ * Fprop, Dgrad, Wgrad and MoE grouped Fprop.
+ *
+ * Sources (web pages reproducing the DeepSeek-V3 report's FP8 training
+ * section; cited by page title, or by host where the page has no title, and
+ * by the figure or passage):
+ *   [P1] "5 Ways You can get More Deepseek While Spending Less"
+ *        (xn--jj0bz6z98ct0a29q.com) -- power-of-2 scaling factors; max-abs
+ *        mapped to the FP8 maximum; per-group scaling along the GEMM inner
+ *        dimension; promotion every 128 elements (four WGMMAs) to FP32 on
+ *        CUDA cores; Figure 6 (Fprop, Dgrad, Wgrad in FP8); 1x128 FP8 tiles
+ *        cached for backward; K = 4096 limited-accumulation error.
+ *   [P2] why-be.co.kr board post -- Figure 7 (a): 1x128 activation tiles and
+ *        128x128 weight blocks; promotion to FP32 registers.
+ *   [P3] cameseeing.com community post -- Figure 7 (a); max-abs computed
+ *        online per 1x128 tile / 128x128 block, scale derived, cast online.
+ *   [P4] "Three Fast Methods To Study Deepseek" -- E4M3 on all tensors;
+ *        Figure 7 (a); MoE layer shapes (expert hidden size 2048, top-8).
+ *   [P5] gnrental.net free-board post -- GEMMs take FP8 inputs and give BF16
+ *        or FP32 outputs; two WGMMAs in flight so promotion overlaps MMA;
+ *        128 BF16 activations read from HBM, FP8 written back, read again.
+ *
+ * Conventions shared by every entry point
+ *   - Every tensor pointer is caller-owned DEVICE memory on the current CUDA
+ *     device (e.g. PyTorch-allocated).  The library allocates nothing and
+ *     keeps no per-call state; its only global state is one status word per
+ *     device (a __device__ variable) and a host-side wait time limit.
+ *   - All calls are asynchronous on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream).  None synchronises except fp8_get_status().
+ *   - Arguments are validated on the host before anything is launched; on a
+ *     validation error the call returns its code, launches nothing and
+ *     writes nothing.  Launch failures return FP8_ERR_LAUNCH.
+ *   - Errors found on the device (a bounded wait that ran out, malformed
+ *     group offsets) are recorded in the status word; read and clear it with
+ *     fp8_get_status().
+ *   - Outputs must not alias inputs.  Pointers must be 16-byte aligned and
+ *     leading dimensions multiples of 16 bytes.
+ *   - Entry points are reentrant; concurrent calls on different streams are
+ *     safe as long as their outputs do not overlap.
+ *   - E4M3 is OCP E4M3FN: 1 sign, 4 exponent (bias 7), 3 mantissa bits; max
+ *     finite 448; codes are stored one per byte.
+ */
+#ifndef FP8FG_H
+#define FP8FG_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. */
+enum fp8_status {
+    FP8_OK = 0,
+    FP8_ERR_NULL = 1,     /* a required pointer is NULL                          */
+    FP8_ERR_SHAPE = 2,    /* size <= 0 where not allowed, not a multiple of 128,
+                             overflow, ld too small, bad group offsets (device)  */
+    FP8_ERR_ALIGN = 3,    /* pointer or leading dimension not 16-byte aligned    */
+    FP8_ERR_DTYPE = 4,    /* unknown dtype / mode / major / granularity enum     */
+    FP8_ERR_LAUNCH = 5,   /* the CUDA launch failed (cudaGetLastError)           */
+    FP8_ERR_TIMEOUT = 6,  /* a bounded device-side wait gave up (status word)    */
+    FP8_ERR_DEVICE = 7    /* no CUDA device, or not an sm_100 (B200-class) GPU   */
+};
+
+enum { FP8_IN_BF16 = 0, FP8_IN_FP32 = 1 };          /* quantizer input dtype   */
+enum { FP8_OUT_BF16 = 0, FP8_OUT_FP32 = 1 };        /* GEMM output dtype       */
+enum { FP8_SCALE_FP32 = 0, FP8_SCALE_POW2 = 1 };    /* scale mode              */
+enum { FP8_B_KMAJOR = 0, FP8_B_MNMAJOR = 1 };       /* layout of GEMM operand B */
+
+/*
+ * Group scale (all three quantizers), per group of 128 or 128x128 elements
+ * with max-abs `amax` ([P1] max-abs -> FP8 max; [P3] online max-abs):
+ *   FP8_SCALE_FP32: s = fl32(amax / 448); codes E(fl32(x * fl32(448 / amax))).
+ *                   amax == 0 gives s = 1 (codes +-0); amax < 1.75*2^-118
+ *                   (amax/448 below FLT_MIN) gives s = 2^-126, codes E(x*2^126).
+ *   FP8_SCALE_POW2: s = 2^e, e the least integer with amax <= 448 * 2^e,
+ *                   clamped to e >= -126 ([P1] integral power-of-2 scales);
+ *                   codes E(x * 2^-e), exact scaling.  amax == 0 gives s = 1.
+ * E() rounds to nearest even and saturates to +-448.  Dequantisation is
+ * code * s.
+ */
+
+/*
+ * 1x128 activation tiles: one scale per token (row) per 128 consecutive
+ * channels ([P2]/[P3]/[P4] Figure 7 (a); [P1] FP8 tiles cached for backward).
+ *   x    [M][ldx] input, row-major, dtype in_dtype (BF16 or FP32)
+ *   q    [M][ldq] E4M3 codes (uint8), same positions as x
+ *   sA   [K/128][M] FP32 scales, sA[kb*M + m] for x[m][kb*128 .. +127]
+ *        ("K-block-major": the M scales of one K-block are contiguous)
+ * Sizes: M >= 0 (M == 0 launches nothing), K > 0 and K % 128 == 0,
+ * ldx >= K, ldq >= K.
+ */
+int fp8_quant_act_1x128(const void* x, int in_dtype, int64_t M, int64_t K, int64_t ldx,
+                        uint8_t* q, int64_t ldq, float* sA, int scale_mode, void* stream);
+
+/*
+ * 128x1 tiles along tokens for the Wgrad operands: one scale per channel
+ * per 128 consecutive tokens, so that the groups run along the Wgrad GEMM's
+ * inner dimension (tokens) as [P1] asks of every FP8 GEMM operand.  The
+ * output is written transposed so the token axis is contiguous (K-major
+ * operand of fp8_blockscaled_gemm).
+ *   x    [T][ldx] input (token-major), BF16 or FP32
+ *   qT   [C][ldqT] E4M3 codes, qT[c][t] is the code of x[t][c]
+ *   s    [T/128][C] FP32 scales, s[tb*C + c] for x[tb*128 .. +127][c]
+ * Sizes: T > 0 and T % 128 == 0; C >= 0 and C % 8 == 0 (C == 0 launches
+ * nothing); ldx >= C, ldqT >= T.
+ */
+int fp8_quant_act_128x1(const void* x, int in_dtype, int64_t T, int64_t C, int64_t ldx,
+                        uint8_t* qT, int64_t ldqT, float* s, int scale_mode, void* stream);
+
+/*
+ * 128x128 weight blocks: one scale per 128 output x 128 input channels
+ * ([P2]/[P3]/[P4] Figure 7 (a)).
+ *   w    [N][ldw] input, row-major, BF16 or FP32
+ *   q    [N][ldq] E4M3 codes
+ *   sW   [N/128][K/128] FP32 scales, sW[nb*(K/128) + kb]
+ * Sizes: N >= 0, N % 128 == 0; K > 0, K % 128 == 0; ldw >= K, ldq >= K.
+ */
+int fp8_quant_w_128x128(const void* w, int in_dtype, int64_t N, int64_t K, int64_t ldw,
+                        uint8_t* q, int64_t ldq, float* sW, int scale_mode, void* stream);
+
+/*
+ * Block-scaled FP8 GEMM  D[m][n] = sum_kb sA[kb][m] * sB(n, kb) * P(m, n, kb)
+ * with P the E4M3 x E4M3 dot product over K-block kb (128 elements) computed
+ * on the tensor cores and promoted to an FP32 running sum every 128 K
+ * ([P1]/[P2]/[P5] increased-precision accumulation, N_C = 128; [P1]
+ * per-group scales along the inner dimension; [P5] FP8 in, BF16/FP32 out;
+ * [P1] Figure 6: used for Fprop, Dgrad and Wgrad).
+ *   A    [M][K] E4M3, row-major (K contiguous)
+ *   sA   [K/128][M] FP32 (as written by fp8_quant_act_1x128 / _128x1)
+ *   B    b_major == FP8_B_KMAJOR : [N][K] E4M3 (K contiguous), e.g. the
+ *                                   quantized weight W[N][K] in Fprop or a
+ *                                   128x1-quantized qT in Wgrad;
+ *        b_major == FP8_B_MNMAJOR: [K][N] E4M3 (N contiguous), e.g. the
+ *                                   forward weight W[K][N] read transposed
+ *                                   in Dgrad ([P5] transposed operand reads)
+ *   sB   sb_gran == 128: 128x128 block scales of the stored B:
+ *                        K-major [N/128][K/128], MN-major [K/128][N/128];
+ *        sb_gran == 1  : per-column scales [K/128][N] (K-major B only)
+ *   D    [M][ldd] row-major, BF16 (round to nearest even) or FP32
+ * Sizes: M >= 0 (0 launches nothing); N > 0, N % 128 == 0; K > 0,
+ * K % 128 == 0; ldd >= N.
+ */
+int fp8_blockscaled_gemm(const uint8_t* A, const float* sA, const uint8_t* B, int b_major,
+                         const float* sB, int sb_gran, int64_t M, int64_t N, int64_t K, void* D,
+                         int out_dtype, int64_t ldd, void* stream);
+
+/*
+ * Grouped (MoE expert) block-scaled GEMM: rows [off[e], off[e+1]) of A are
+ * multiplied by expert e's weight ([P4] MoE layer; [P5] each group only
+ * loads the parameters of one expert).
+ *   A        [M_total][K] E4M3, rows grouped by expert, zero rows as padding
+ *   sA       [K/128][M_total] FP32
+ *   B        [G][N][K] E4M3 (K-major per expert)
+ *   sB       [G][N/128][K/128] FP32
+ *   group_offsets  [G+1] int32 in DEVICE memory: off[0] == 0, non-decreasing,
+ *            every entry a multiple of 128, off[G] <= M_total.  Empty groups
+ *            are allowed.  Checked on the device: malformed offsets record
+ *            FP8_ERR_SHAPE in the status word and nothing is written.
+ *   D        [M_total][N] (row stride N), BF16 or FP32; rows at or beyond
+ *            off[G] are left untouched.
+ * Sizes: G >= 1; M_total >= 0 and M_total % 128 == 0; N > 0, N % 128 == 0;
+ * K > 0, K % 128 == 0.
+ */
+int fp8_grouped_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB,
+                     const int32_t* group_offsets, int G, int64_t M_total, int64_t N, int64_t K,
+                     void* D, int out_dtype, void* stream);
+
+/*
+ * Synchronise `stream`, then return and clear the current device's status
+ * word (FP8_OK if no kernel reported an error since the last call).  Returns
+ * FP8_ERR_DEVICE if the status cannot be read.
+ */
+int fp8_get_status(void* stream);
+
+/* Human-readable name of a return code (static string, never NULL). */
+const char* fp8_status_string(int code);
+
+/*
+ * Time limit, in nanoseconds, of every device-side wait of kernels launched
+ * after this call (default 4e9).  0 restores the default.  Not thread-safe
+ * with respect to concurrent launches; meant for tests and debugging.
+ */
+void fp8_set_wait_timeout_ns(uint64_t ns);
+
+/*
+ * Self-test of the bounded-wait machinery: launches one CTA that waits on an
+ * mbarrier nothing ever arrives at, with the current time limit.  The kernel
+ * gives up after the limit, records FP8_ERR_TIMEOUT and returns normally, so
+ * fp8_get_status() afterwards reports FP8_ERR_TIMEOUT and the context stays
+ * usable.  Returns FP8_OK if the launch succeeded.
+ */
+int fp8_selftest_wait_timeout(void* stream);
+
+/* 1 if the current device is an sm_100 GPU the library runs on, else 0. */
+int fp8_device_supported(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8FG_H */

@@ -1,0 +1,145 @@
+"""Full-size parity of the five workloads, run exactly as bench.py runs them
+(the step objects of fp8_fine_grained_x1_b200.linear, one GPU, persistent
+GEMM grid), against the CPU oracle on the same seeded inputs.
+
+Quantized operands are compared in full (bit-exact); GEMM outputs at
+sampled points the oracle computes one by one: 4096 random (m, n), whole
+rows and columns at the first/last tile edges, and for the MoE layer the
+first, last-real and last-padding row of every expert group.
+"""
+import numpy as np
+import pytest
+import torch
+
+import fp8_fine_grained_x1_b200 as fg
+import oracle
+from fp8_fine_grained_x1_b200 import linear, synth
+
+from gpu_util import assert_gemm_close, d2h, dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _points(M, N, seed, n_random=4096, rows=(), cols=()):
+    rng = np.random.default_rng(seed)
+    pts = [np.stack([rng.integers(0, M, n_random), rng.integers(0, N, n_random)], 1)]
+    for m in rows:
+        pts.append(np.stack([np.full(N, m), np.arange(N)], 1))
+    for n in cols:
+        pts.append(np.stack([np.arange(M), np.full(M, n)], 1))
+    return np.concatenate(pts).astype(np.int64)
+
+
+def _edges(n, tile):
+    return sorted({0, min(tile - 1, n - 1), min(tile, n - 1), n - 1})
+
+
+def _bits(t):
+    return synth.bf16_bits(t) if t.dtype == torch.bfloat16 else t.numpy()
+
+
+def test_pr1_tiny_fprop_full_output():
+    wl = synth.pr1()
+    step = linear.FpropStep(wl["x"].to(dev()), wl["w"].to(dev()), out_dtype=torch.float32)
+    y = d2h(step())
+    assert fg.fp8_get_status() == fg.FP8_OK
+    qx, sx = oracle.quant_act_1x128(wl["x"].numpy())
+    qw, sw = oracle.quant_w_128x128(wl["w"].numpy())
+    assert np.array_equal(step.qx.cpu().numpy(), qx) and np.array_equal(step.sx.cpu().numpy(), sx)
+    assert np.array_equal(step.qw.cpu().numpy(), qw) and np.array_equal(step.sw.cpu().numpy(), sw)
+    ref, tol = oracle.gemm_full(qx, sx, qw, sw)
+    assert_gemm_close(y, ref, tol, False, "pr1")
+
+
+def test_fprop_dense_mlp():
+    wl = synth.fprop()
+    step = linear.FpropStep(wl["x"].to(dev()), wl["w"].to(dev()))
+    y = step()
+    torch.cuda.synchronize()
+    assert fg.fp8_get_status() == fg.FP8_OK
+    qx, sx = oracle.quant_act_1x128(_bits(wl["x"]))
+    qw, sw = oracle.quant_w_128x128(_bits(wl["w"]))
+    assert np.array_equal(step.qx.cpu().numpy(), qx) and np.array_equal(step.sx.cpu().numpy(), sx)
+    assert np.array_equal(step.qw.cpu().numpy(), qw) and np.array_equal(step.sw.cpu().numpy(), sw)
+    M, N = y.shape
+    pts = _points(M, N, 1, rows=_edges(M, 128), cols=_edges(N, 256))
+    ref, tol = oracle.gemm_points(qx, sx, qw, sw, pts)
+    got = d2h(y)[pts[:, 0], pts[:, 1]]
+    assert_gemm_close(got, ref, tol, True, "fprop")
+
+
+def test_dgrad_reads_weight_transposed():
+    wl = synth.dgrad()
+    step = linear.DgradStep(wl["dy"].to(dev()), wl["w"].to(dev()))
+    dx = step()
+    torch.cuda.synchronize()
+    assert fg.fp8_get_status() == fg.FP8_OK
+    qdy, sdy = oracle.quant_act_1x128(_bits(wl["dy"]))
+    qw, sw = oracle.quant_w_128x128(_bits(wl["w"]))               # stored [N_out][K_in]
+    assert np.array_equal(step.qdy.cpu().numpy(), qdy) and np.array_equal(step.qw.cpu().numpy(), qw)
+    M, N = dx.shape
+    pts = _points(M, N, 2, rows=_edges(M, 128), cols=_edges(N, 256))
+    ref, tol = oracle.gemm_points(qdy, sdy, qw, sw, pts, b_major=oracle.B_MNMAJOR)
+    assert_gemm_close(d2h(dx)[pts[:, 0], pts[:, 1]], ref, tol, True, "dgrad")
+
+
+@pytest.mark.parametrize("mode", [fg.SCALE_FP32, fg.SCALE_POW2])
+def test_wgrad_token_axis_groups(mode):
+    wl = synth.wgrad()
+    step = linear.WgradStep(wl["x"].to(dev()), wl["dy"].to(dev()), scale_mode=mode)
+    dw = step()
+    torch.cuda.synchronize()
+    assert fg.fp8_get_status() == fg.FP8_OK
+    qxT, sx = oracle.quant_act_128x1(_bits(wl["x"]), mode)
+    qdyT, sdy = oracle.quant_act_128x1(_bits(wl["dy"]), mode)
+    assert np.array_equal(step.qxT.cpu().numpy(), qxT) and np.array_equal(step.sx.cpu().numpy(), sx)
+    assert np.array_equal(step.qdyT.cpu().numpy(), qdyT) and np.array_equal(step.sdy.cpu().numpy(), sdy)
+    M, N = dw.shape
+    pts = _points(M, N, 3, rows=_edges(M, 128), cols=_edges(N, 256))
+    ref, tol = oracle.gemm_points(qdyT, sdy, qxT, sx, pts, sb_gran=1)
+    assert_gemm_close(d2h(dw)[pts[:, 0], pts[:, 1]], ref, tol, False, f"wgrad mode={mode}")
+
+
+def test_moe_grouped_fprop():
+    wl = synth.moe()
+    lay = wl["layout"]
+    a = synth.gather_rows(wl["x"].to(dev()), lay.row_token)
+    G, N, K = wl["w"].shape
+    off = lay.offsets.numpy()
+    step = linear.MoeStep(a, wl["w"].to(dev()), lay.offsets.to(dev()))
+    y = step()
+    torch.cuda.synchronize()
+    assert fg.fp8_get_status() == fg.FP8_OK
+
+    # weights: every expert, bit-exact
+    qw, sw = oracle.quant_w_128x128(_bits(wl["w"].view(G * N, K)))
+    assert np.array_equal(step.qw.cpu().numpy().reshape(G * N, K), qw)
+    assert np.array_equal(step.sw.cpu().numpy().reshape(G * N // 128, K // 128), sw)
+    qw = qw.reshape(G, N, K)
+    sw = sw.reshape(G, N // 128, K // 128)
+
+    # sampled rows: group edges (first, last real, last padding) + random rows
+    rng = np.random.default_rng(4)
+    rows = set(rng.integers(0, lay.m_total, 64).tolist())
+    for e in range(G):
+        if off[e + 1] > off[e]:
+            rows |= {int(off[e]), int(off[e] + lay.counts[e] - 1), int(off[e + 1] - 1)}
+    rows = np.array(sorted(rows))
+    tok = lay.row_token[rows]
+    a_rows = synth.gather_rows(wl["x"], tok)                       # CPU, same rows
+    qa_r, sa_r = oracle.quant_act_1x128(_bits(a_rows))
+    assert np.array_equal(step.qa[torch.from_numpy(rows).to(dev())].cpu().numpy(), qa_r)
+    assert np.array_equal(step.sa[:, torch.from_numpy(rows).to(dev())].cpu().numpy(), sa_r)
+
+    yh = d2h(y)
+    for e in range(G):
+        sel = np.flatnonzero((rows >= off[e]) & (rows < off[e + 1]))
+        if sel.size == 0:
+            continue
+        pts = np.array([(i, n) for i in sel for n in range(N)], np.int64)
+        ref, tol = oracle.gemm_points(qa_r, sa_r, qw[e], sw[e], pts)
+        got = yh[rows[pts[:, 0]], pts[:, 1]]
+        assert_gemm_close(got, ref, tol, True, f"moe expert {e}")
+    # padding rows are exactly zero
+    pad = lay.row_token.numpy() < 0
+    assert np.all(yh[pad] == 0.0)
