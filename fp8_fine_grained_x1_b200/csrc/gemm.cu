@@ -28,6 +28,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <cstddef>
 #include <cstdint>
 #include <mutex>
 
@@ -107,7 +108,9 @@ __device__ __forceinline__ int find_group(const int32_t* off, int G, int64_t row
     return lo < G ? lo : -1;
 }
 
-struct Shared {
+struct __align__(16) Shared {
+    float sbw[NUM_PROMO_WARPS][2][128];   // per-warp column scales (sb_gran == 1),
+                                          // read and written as float4: first, 16-B aligned
     uint64_t full[NS];
     uint64_t empty[NS];
     uint64_t tfull[2];
@@ -117,8 +120,10 @@ struct Shared {
     int abort;
     int bad;
     int32_t off[MAX_GROUPS + 1];
-    float sbw[NUM_PROMO_WARPS][2][128];   // per-warp column scales (sb_gran == 1)
 };
+static_assert(offsetof(Shared, sbw) % 16 == 0, "float4 accesses need 16-byte alignment");
+static_assert(sizeof(float) * 128 % 16 == 0, "per-warp scale rows stay 16-byte aligned");
+static_assert(offsetof(Shared, full) % 8 == 0, "mbarriers need 8-byte alignment");
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
