@@ -70,6 +70,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
     return ok != 0;
 }
 
+// Same test, but a thread whose phase is not complete is suspended in hardware
+// (for at most `hint_ns`) until it completes, instead of returning at once:
+// a waiting warp then leaves its scheduler's issue slots to the other warps.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+constexpr uint32_t kWaitSleepNs = 20000;   // per suspended try_wait (bounded loop below)
+
 // Wait until the phase of `bar` with parity `parity` has completed.
 // Gives up (returns false) when *abort is set by another role of the CTA or
 // when `timeout_ns` has passed; in the latter case it records
@@ -81,11 +99,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1; it < (1u << 30); ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63) == 0) {
-            if (*abort) return false;
-            if (globaltimer_ns() - t0 > timeout_ns) break;
-        }
+        if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
+        if (*abort) return false;
+        if ((it & 7) == 0 && globaltimer_ns() - t0 > timeout_ns) break;
     }
     report_error(FP8_ERR_TIMEOUT);
     *abort = 1;
@@ -99,8 +115,8 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, 
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1; it < (1u << 30); ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63) == 0 && globaltimer_ns() - t0 > timeout_ns) break;
+        if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
+        if ((it & 7) == 0 && globaltimer_ns() - t0 > timeout_ns) break;
     }
     report_error(FP8_ERR_TIMEOUT);
     return false;
