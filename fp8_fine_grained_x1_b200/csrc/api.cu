@@ -63,7 +63,7 @@ FP8FG_API int fp8_quant_act_1x128(const void* x, int in_dtype, int64_t M, int64_
                                   uint8_t* q, int64_t ldq, float* sA, int scale_mode, void* stream)
 {
     if (!is_in(in_dtype) || !is_mode(scale_mode)) return FP8_ERR_DTYPE;
-    if (M < 0 || M > kMaxDim || K <= 0 || K > kMaxDim || K % 128 || K / 128 > 65535 || ldx < K ||
+    if (M < 0 || M > kMaxDim || (M + 127) / 128 > 65535 || K <= 0 || K > kMaxDim || K % 128 || ldx < K ||
         ldq < K || ldx > kMaxDim || ldq > kMaxDim)
         return FP8_ERR_SHAPE;
     if (M == 0) return FP8_OK;

@@ -137,11 +137,14 @@ __device__ __forceinline__ float absmax8(const float (&v)[8])
 
 // ------------------------------------------------------------ 1x128
 
-constexpr int kRowsPerCta1x128 = 64;   // 16 groups in flight x 4 per thread
+constexpr int kGroupsPerThread1x128 = 8;
+constexpr int kRowsPerCta1x128 = 16 * kGroupsPerThread1x128;   // 128
 
 // CTA = 256 threads = 16 half-warps; a half-warp owns one 1x128 group at a
-// time (16 lanes x 8 elements); each thread keeps 4 groups' loads in flight.
-// Grid: x = ceil(M/64) row blocks, y = K/128 K-blocks.
+// time (16 lanes x 8 elements); each thread keeps 8 groups' loads (128 B) in
+// flight before reducing any of them.
+// Grid: x = K/128 K-blocks (adjacent CTAs read adjacent 256-byte segments of
+// the same rows), y = ceil(M/128) row blocks.
 template <typename Tin>
 __global__ void __launch_bounds__(256) k_quant_1x128(const Tin* __restrict__ x, int64_t M,
                                                      int64_t ldx, uint8_t* __restrict__ q,
@@ -149,12 +152,12 @@ __global__ void __launch_bounds__(256) k_quant_1x128(const Tin* __restrict__ x, 
 {
     const int h = threadIdx.x >> 4;
     const int l = threadIdx.x & 15;
-    const int64_t kb = blockIdx.y;
-    const int64_t m0 = (int64_t)blockIdx.x * kRowsPerCta1x128;
+    const int64_t kb = blockIdx.x;
+    const int64_t m0 = (int64_t)blockIdx.y * kRowsPerCta1x128;
 
-    Chunk8<Tin> c[4];
+    Chunk8<Tin> c[kGroupsPerThread1x128];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kGroupsPerThread1x128; ++u) {
         const int64_t m = m0 + u * 16 + h;
         if (m < M)
             c[u].load(x + m * ldx + kb * 128 + l * 8);
@@ -162,7 +165,7 @@ __global__ void __launch_bounds__(256) k_quant_1x128(const Tin* __restrict__ x, 
             c[u].zero();
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kGroupsPerThread1x128; ++u) {
         const int64_t m = m0 + u * 16 + h;
         float v[8];
         c[u].get(v);
@@ -234,74 +237,134 @@ __global__ void __launch_bounds__(256) k_quant_w128(const Tin* __restrict__ w, i
 
 // ------------------------------------------------------------ 128x1
 
-constexpr int kTok = 128;   // tokens per tile (one group along tokens)
-constexpr int kCh = 64;     // channels per tile
-
-// CTA = 256 threads per tile of 128 tokens x 64 channels.  The tile is staged
-// in shared memory with coalesced 16-byte row loads; then thread
-// (c = tid%64, quarter = tid/64) walks 32 tokens of channel c, the four
-// quarters combine their max-abs, and each thread writes its 32 codes as two
-// 16-byte stores into the transposed output row qT[c].
-// Grid: x = ceil(C/64), y = T/128.
+constexpr int kTok = 128;        // tokens per tile (one group along tokens)
+constexpr int kThr128x1 = 256;
+// Tile geometry per input type: 128-byte row segments (64 BF16 or 32 FP32
+// channels), threads own channel pairs x (kTok / kGroups) tokens.  (256-byte
+// segments with 512 threads measured slower.)
 template <typename Tin>
-__global__ void __launch_bounds__(256) k_quant_128x1(const Tin* __restrict__ x, int64_t C,
-                                                     int64_t ldx, uint8_t* __restrict__ qT,
-                                                     int64_t ldqT, float* __restrict__ s, int mode)
+struct Geo128x1 {
+    static constexpr int kCh = 128 / (int)sizeof(Tin);
+    static constexpr int kPairs = kCh / 2;
+    static constexpr int kGroups = kThr128x1 / kPairs;   // 8 (BF16) or 16 (FP32)
+    static constexpr int kTokPerThr = kTok / kGroups;    // 16 (BF16) or 8 (FP32)
+    static_assert(kTokPerThr == 16 || kTokPerThr == 8, "16- or 8-byte code stores");
+};
+
+// CTA = 256 threads per tile of 128 tokens x 128 bytes of channels (64 BF16
+// or 32 FP32 channels).  The tile is staged
+// in shared memory with register-free 16-byte cp.async copies (coalesced row
+// segments), so registers do not limit how many tiles are in flight per SM.
+// Thread (p = tid % kPairs, g = tid / kPairs) then owns channels 2p, 2p+1 and
+// kTokPerThr tokens starting at g * kTokPerThr, read as two-channel words (a
+// warp reads 128 or 256 contiguous bytes of one row per load, conflict-free):
+// a first pass takes the max-abs, the token groups combine theirs through
+// shared memory, and a second pass encodes the thread's tokens of each
+// channel into one 16- or 8-byte store per channel of the transposed output.
+// Grid: x = ceil(C / kCh), y = T/128.
+template <typename Tin>
+struct Pair;
+template <>
+struct Pair<__nv_bfloat16> {
+    // two adjacent bf16 channels of one token as one 32-bit word
+    static __device__ __forceinline__ float2 get(const __nv_bfloat16* p)
+    {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
+        return make_float2(bf16_lo(w), bf16_hi(w));
+    }
+};
+template <>
+struct Pair<float> {
+    static __device__ __forceinline__ float2 get(const float* p) { return *reinterpret_cast<const float2*>(p); }
+};
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc)
 {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(kThr128x1, 6) k_quant_128x1(const Tin* __restrict__ x, int64_t C,
+                                                              int64_t ldx, uint8_t* __restrict__ qT,
+                                                              int64_t ldqT, float* __restrict__ s, int mode)
+{
+    using G = Geo128x1<Tin>;
     constexpr int kElemsPerChunk = 16 / (int)sizeof(Tin);
-    constexpr int kChunksPerRow = kCh / kElemsPerChunk;
-    constexpr int kChunksPerThread = kTok * kChunksPerRow / 256;
-    __shared__ __align__(16) Tin tile[kTok][kCh];
-    __shared__ float part[4][kCh];
+    constexpr int kChunksPerRow = G::kCh / kElemsPerChunk;           // 8
+    constexpr int kChunksPerThread = kTok * kChunksPerRow / kThr128x1;   // 4
+    __shared__ __align__(16) Tin tile[kTok][G::kCh];
+    __shared__ float2 part[G::kGroups][G::kPairs];
 
     const int64_t tb = blockIdx.y;
-    const int64_t c0 = (int64_t)blockIdx.x * kCh;
+    const int64_t c0 = (int64_t)blockIdx.x * G::kCh;
 
     // 1. stage the tile (channels beyond C are zero; C % 8 == 0)
-    uint4 buf[kChunksPerThread];
 #pragma unroll
     for (int i = 0; i < kChunksPerThread; ++i) {
-        const int id = threadIdx.x + 256 * i;
+        const int id = threadIdx.x + kThr128x1 * i;
         const int r = id / kChunksPerRow;
         const int j = id % kChunksPerRow;
         const int64_t ch = c0 + j * kElemsPerChunk;
-        buf[i] = (ch < C) ? ld_stream16(x + (tb * kTok + r) * ldx + ch) : make_uint4(0, 0, 0, 0);
+        if (ch < C)
+            cp_async16(&tile[r][j * kElemsPerChunk], x + (tb * kTok + r) * ldx + ch);
+        else
+            *reinterpret_cast<uint4*>(&tile[r][j * kElemsPerChunk]) = make_uint4(0, 0, 0, 0);
     }
-#pragma unroll
-    for (int i = 0; i < kChunksPerThread; ++i) {
-        const int id = threadIdx.x + 256 * i;
-        const int r = id / kChunksPerRow;
-        const int j = id % kChunksPerRow;
-        *reinterpret_cast<uint4*>(&tile[r][j * kElemsPerChunk]) = buf[i];
-    }
+    cp_async_wait_all();
     __syncthreads();
 
-    // 2. column max-abs over 4 x 32 tokens
-    const int c = threadIdx.x % kCh;
-    const int qtr = threadIdx.x / kCh;
-    float v[32];
-    float a = 0.0f;
+    // 2. max-abs of channels 2p, 2p+1 over this thread's tokens, then over groups
+    const int pch = threadIdx.x % G::kPairs;
+    const int g = threadIdx.x / G::kPairs;
+    const int t0 = g * G::kTokPerThr;
+    float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
-    for (int t = 0; t < 32; ++t) {
-        v[t] = (float)tile[qtr * 32 + t][c];
-        a = fmaxf(a, fabsf(v[t]));
+    for (int t = 0; t < G::kTokPerThr; ++t) {
+        const float2 v = Pair<Tin>::get(&tile[t0 + t][2 * pch]);
+        a0 = fmaxf(a0, fabsf(v.x));
+        a1 = fmaxf(a1, fabsf(v.y));
     }
-    part[qtr][c] = a;
+    part[g][pch] = make_float2(a0, a1);
     __syncthreads();
-    a = fmaxf(fmaxf(part[0][c], part[1][c]), fmaxf(part[2][c], part[3][c]));
-    const GroupScale g = group_scale(a, mode);
-
-    // 3. encode 32 tokens of channel c, store transposed
-    const int64_t ch = c0 + c;
-    if (ch < C) {
-        uint32_t w[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            w[i] = encode4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3], g.inv);
-        uint4* dst = reinterpret_cast<uint4*>(qT + ch * ldqT + tb * kTok + qtr * 32);
-        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-        if (qtr == 0) s[tb * C + ch] = g.s;
+    for (int i = 0; i < G::kGroups; ++i) {
+        const float2 q = part[i][pch];
+        a0 = fmaxf(a0, q.x);
+        a1 = fmaxf(a1, q.y);
+    }
+    const GroupScale g0 = group_scale(a0, mode);
+    const GroupScale g1 = group_scale(a1, mode);
+
+    // 3. encode this thread's tokens of each channel, store transposed
+    const int64_t ch = c0 + 2 * pch;
+    if (ch < C) {   // C % 8 == 0: ch < C implies ch + 1 < C
+        uint32_t w0[G::kTokPerThr / 4], w1[G::kTokPerThr / 4];
+#pragma unroll
+        for (int q4 = 0; q4 < G::kTokPerThr / 4; ++q4) {
+            float2 v[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) v[t] = Pair<Tin>::get(&tile[t0 + q4 * 4 + t][2 * pch]);
+            w0[q4] = encode4(v[0].x, v[1].x, v[2].x, v[3].x, g0.inv);
+            w1[q4] = encode4(v[0].y, v[1].y, v[2].y, v[3].y, g1.inv);
+        }
+        uint8_t* d0 = qT + ch * ldqT + tb * kTok + t0;
+        uint8_t* d1 = d0 + ldqT;
+        if constexpr (G::kTokPerThr == 16) {
+            *reinterpret_cast<uint4*>(d0) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+            *reinterpret_cast<uint4*>(d1) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+        } else {
+            *reinterpret_cast<uint2*>(d0) = make_uint2(w0[0], w0[1]);
+            *reinterpret_cast<uint2*>(d1) = make_uint2(w1[0], w1[1]);
+        }
+        if (g == 0) {   // s is only guaranteed 4-byte aligned: two scalar stores
+            s[tb * C + ch] = g0.s;
+            s[tb * C + ch + 1] = g1.s;
+        }
     }
 }
 
@@ -312,7 +375,7 @@ __global__ void __launch_bounds__(256) k_quant_128x1(const Tin* __restrict__ x, 
 cudaError_t launch_quant_act_1x128(const void* x, int in_dtype, int64_t M, int64_t K, int64_t ldx,
                                    uint8_t* q, int64_t ldq, float* sA, int mode, cudaStream_t st)
 {
-    const dim3 grid((unsigned)((M + kRowsPerCta1x128 - 1) / kRowsPerCta1x128), (unsigned)(K / 128));
+    const dim3 grid((unsigned)(K / 128), (unsigned)((M + kRowsPerCta1x128 - 1) / kRowsPerCta1x128));
     if (in_dtype == FP8_IN_BF16)
         k_quant_1x128<__nv_bfloat16><<<grid, 256, 0, st>>>(
             static_cast<const __nv_bfloat16*>(x), M, ldx, q, ldq, sA, mode);
@@ -325,12 +388,13 @@ cudaError_t launch_quant_act_1x128(const void* x, int in_dtype, int64_t M, int64
 cudaError_t launch_quant_act_128x1(const void* x, int in_dtype, int64_t T, int64_t C, int64_t ldx,
                                    uint8_t* qT, int64_t ldqT, float* s, int mode, cudaStream_t st)
 {
-    const dim3 grid((unsigned)((C + kCh - 1) / kCh), (unsigned)(T / kTok));
+    const int ch_tile = in_dtype == FP8_IN_BF16 ? Geo128x1<__nv_bfloat16>::kCh : Geo128x1<float>::kCh;
+    const dim3 grid((unsigned)((C + ch_tile - 1) / ch_tile), (unsigned)(T / kTok));
     if (in_dtype == FP8_IN_BF16)
-        k_quant_128x1<__nv_bfloat16><<<grid, 256, 0, st>>>(
+        k_quant_128x1<__nv_bfloat16><<<grid, kThr128x1, 0, st>>>(
             static_cast<const __nv_bfloat16*>(x), C, ldx, qT, ldqT, s, mode);
     else
-        k_quant_128x1<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), C, ldx, qT,
+        k_quant_128x1<float><<<grid, kThr128x1, 0, st>>>(static_cast<const float*>(x), C, ldx, qT,
                                                    ldqT, s, mode);
     return cudaGetLastError();
 }
