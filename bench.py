@@ -200,15 +200,20 @@ def make_step(workload, device):
     elif workload == "moe":
         wl = synth.moe()
         lay = wl["layout"]
-        a = synth.gather_rows(wl["x"].to(device), lay.row_token)
-        step = linear.MoeStep(a, wl["w"].to(device), lay.offsets.to(device))
+        topk = lay.topk.to(torch.int32)
+        step = linear.MoeStep(wl["x"].to(device), topk.to(device), wl["w"].to(device))
         G, N, K = wl["w"].shape
+        T = wl["x"].shape[0]
         M = int(lay.counts.sum())
         desc = dict(workload="moe grouped fprop, 32 experts W_e[2048,7168], 16384 tokens "
-                    "top-8 Zipf(1.1), groups padded to 128, bf16 out", M=M, N=N, K=K,
-                    M_padded=lay.m_total)
-        inputs = [a.cpu(), wl["w"]]
-        quant_bytes = (lay.m_total * K + G * N * K) * 3 + (lay.m_total * K // 128) * 4
+                    "top-8 Zipf(1.1): 1x128 quantize tokens, FP8 dispatch to 128-padded "
+                    "groups, 128x128 quantize weights, grouped GEMM, bf16 out",
+                    M=M, N=N, K=K, M_padded=lay.m_total, tokens=T)
+        inputs = [wl["x"], wl["w"], topk]
+        # tokens read once (2 B) + codes written (1 B); dispatched codes read
+        # once per token (1 B) and written per padded row (1 B); weights 3 B
+        quant_bytes = (T * K * 3 + T * K // 32 + (T + lay.m_total) * K + lay.m_total * K // 32
+                       + G * N * K * 3)
     else:
         raise SystemExit(f"unknown workload {workload}")
     flops = 2 * M * N * K
@@ -446,7 +451,7 @@ def _step_inputs(step):
         return [step.dy, step.w]
     if isinstance(step, linear.WgradStep):
         return [step.x, step.dy]
-    return [step.a, step.w]
+    return [step.x, step.w, step.topk]
 
 
 def _step_output(step):

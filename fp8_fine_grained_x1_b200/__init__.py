@@ -43,6 +43,7 @@ EXPORTED = (
     "fp8_quant_act_1x128", "fp8_quant_act_128x1", "fp8_quant_w_128x128",
     "fp8_blockscaled_gemm", "fp8_grouped_gemm", "fp8_get_status", "fp8_status_string",
     "fp8_set_wait_timeout_ns", "fp8_selftest_wait_timeout", "fp8_device_supported",
+    "fp8_moe_dispatch_workspace_bytes", "fp8_moe_dispatch", "fp8_moe_combine",
 )
 
 
@@ -85,6 +86,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fp8_selftest_wait_timeout.restype = _I
     lib.fp8_device_supported.argtypes = []
     lib.fp8_device_supported.restype = _I
+    lib.fp8_moe_dispatch_workspace_bytes.argtypes = [_I64, _I, _I]
+    lib.fp8_moe_dispatch_workspace_bytes.restype = _I64
+    lib.fp8_moe_dispatch.argtypes = [_P, _P, _I64, _I64, _P, _I, _I, _P, _P, _I64, _P, _P, _P,
+                                     _P, _I64, _P]
+    lib.fp8_moe_dispatch.restype = _I
+    lib.fp8_moe_combine.argtypes = [_P, _I, _I64, _I64, _P, _P, _I64, _I, _P, _P]
+    lib.fp8_moe_combine.restype = _I
     _lib = lib
     return lib
 
@@ -177,6 +185,32 @@ def fp8_grouped_gemm(A, sA, B, sB, group_offsets, D, stream=None) -> None:
         _out_dtype(D), _stream(stream)), "fp8_grouped_gemm")
 
 
+def fp8_moe_dispatch_workspace_bytes(T: int, k: int, G: int) -> int:
+    return int(load_library().fp8_moe_dispatch_workspace_bytes(T, k, G))
+
+
+def fp8_moe_dispatch(q, sA, topk, G, q_out, sA_out, group_offsets, token_row, row_token,
+                     workspace, stream=None) -> None:
+    """FP8 rows of the tokens (q [T,K], sA [K/128,T]) to expert-contiguous,
+    128-padded groups (q_out [M_cap,K], sA_out [K/128,M_cap]); topk [T,k] int32."""
+    T, K = q.shape
+    k = topk.shape[1]
+    M_cap = q_out.shape[0]
+    _check(load_library().fp8_moe_dispatch(
+        _ptr(q), _ptr(sA), T, K, _ptr(topk), k, G, _ptr(q_out), _ptr(sA_out), M_cap,
+        _ptr(group_offsets), _ptr(token_row), _ptr(row_token), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)), "fp8_moe_dispatch")
+
+
+def fp8_moe_combine(D, token_row, weights, out, stream=None) -> None:
+    """out[t] = BF16(sum_j weights[t,j] * D[token_row[t,j]]), FP32 sums."""
+    M_cap, N = D.shape
+    T, k = weights.shape
+    _check(load_library().fp8_moe_combine(
+        _ptr(D), _out_dtype(D), M_cap, N, _ptr(token_row), _ptr(weights), T, k, _ptr(out),
+        _stream(stream)), "fp8_moe_combine")
+
+
 def fp8_get_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status word."""
     return load_library().fp8_get_status(_stream(stream))
@@ -231,6 +265,30 @@ def gemm(A, sA, B, sB, out_dtype=None, b_major: int = B_KMAJOR, sb_gran: int = 1
     D = torch.empty((M, N), dtype=out_dtype or torch.bfloat16, device=A.device)
     fp8_blockscaled_gemm(A, sA, B, sB, D, b_major, sb_gran, stream)
     return D
+
+
+def moe_capacity(T: int, k: int, G: int) -> int:
+    """Rows that always hold the padded groups: T*k + G*127, rounded up to 128."""
+    return (T * k + G * 127 + 127) // 128 * 128
+
+
+def moe_dispatch(q, sA, topk, G: int, M_cap: int = None, stream=None):
+    """Allocating form of fp8_moe_dispatch; returns a dict of the outputs."""
+    import torch
+    T, K = q.shape
+    k = topk.shape[1]
+    M_cap = moe_capacity(T, k, G) if M_cap is None else M_cap
+    d = q.device
+    out = dict(q=torch.empty((M_cap, K), dtype=torch.uint8, device=d),
+               sA=torch.empty((K // 128, M_cap), dtype=torch.float32, device=d),
+               offsets=torch.empty(G + 1, dtype=torch.int32, device=d),
+               token_row=torch.empty((T, k), dtype=torch.int32, device=d),
+               row_token=torch.empty(M_cap, dtype=torch.int32, device=d))
+    ws = torch.empty(max(1, fp8_moe_dispatch_workspace_bytes(T, k, G) // 4), dtype=torch.int32,
+                     device=d)
+    fp8_moe_dispatch(q, sA, topk, G, out["q"], out["sA"], out["offsets"], out["token_row"],
+                     out["row_token"], ws, stream)
+    return out
 
 
 def grouped_gemm(A, sA, B, sB, group_offsets, out_dtype=None, stream=None):

@@ -19,6 +19,8 @@ namespace {
 constexpr uint64_t kDefaultTimeoutNs = 4000000000ull;
 std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
 constexpr int64_t kMaxDim = 0x7FFFFFFF;   // sizes and coordinates fit in int32
+// MoE pairs T*k: their padded rows (at most T*k + 1024*127) also fit in int32
+constexpr int64_t kMaxPairs = kMaxDim - 1024 * 128;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 bool is_mode(int m) { return m == FP8_SCALE_FP32 || m == FP8_SCALE_POW2; }
@@ -156,9 +158,60 @@ FP8FG_API int fp8_grouped_gemm(const uint8_t* A, const float* sA, const uint8_t*
                                    D, out_dtype, N, static_cast<cudaStream_t>(stream));
 }
 
+FP8FG_API int64_t fp8_moe_dispatch_workspace_bytes(int64_t T, int k, int G)
+{
+    if (T < 0 || k < 1 || G < 1 || G > 1024 || T > kMaxPairs / k) return 0;
+    return moe_dispatch_workspace_ints(T * k, G) * (int64_t)sizeof(int32_t);
+}
+
+FP8FG_API int fp8_moe_dispatch(const uint8_t* q, const float* sA, int64_t T, int64_t K,
+                               const int32_t* topk, int k, int G, uint8_t* q_out, float* sA_out,
+                               int64_t M_cap, int32_t* group_offsets, int32_t* token_row,
+                               int32_t* row_token, void* workspace, int64_t workspace_bytes,
+                               void* stream)
+{
+    if (T < 0 || K <= 0 || K % 128 || K > kMaxDim || k < 1 || G < 1 || G > 1024 || M_cap < 0 ||
+        M_cap % 128 || M_cap > kMaxDim || T > kMaxPairs / k)
+        return FP8_ERR_SHAPE;
+    if (workspace_bytes < fp8_moe_dispatch_workspace_bytes(T, k, G)) return FP8_ERR_SHAPE;
+    if (!group_offsets || (T > 0 && (!q || !sA || !topk || !token_row || !workspace)) ||
+        (M_cap > 0 && (!q_out || !sA_out || !row_token)))
+        return FP8_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(q_out, 16) || !aligned(sA, 4) || !aligned(sA_out, 4) ||
+        !aligned(topk, 4) || !aligned(group_offsets, 4) || !aligned(token_row, 4) ||
+        !aligned(row_token, 4) || !aligned(workspace, 4))
+        return FP8_ERR_ALIGN;
+    if (!device_is_sm100()) return FP8_ERR_DEVICE;
+    return launch_moe_dispatch(q, sA, T, K, topk, k, G, q_out, sA_out, M_cap, group_offsets,
+                               token_row, row_token, static_cast<int32_t*>(workspace),
+                               static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? FP8_OK
+               : FP8_ERR_LAUNCH;
+}
+
+FP8FG_API int fp8_moe_combine(const void* D, int d_dtype, int64_t M_cap, int64_t N,
+                              const int32_t* token_row, const float* weights, int64_t T, int k,
+                              void* out, void* stream)
+{
+    if (!is_out(d_dtype)) return FP8_ERR_DTYPE;
+    if (T < 0 || T > 0x7FFFFFFF || k < 1 || N <= 0 || N % 8 || N > kMaxDim || M_cap < 0)
+        return FP8_ERR_SHAPE;
+    if (T == 0) return FP8_OK;
+    if (!D || !token_row || !weights || !out) return FP8_ERR_NULL;
+    if (!aligned(D, 16) || !aligned(out, 16) || !aligned(token_row, 4) || !aligned(weights, 4))
+        return FP8_ERR_ALIGN;
+    if (!device_is_sm100()) return FP8_ERR_DEVICE;
+    return launch_moe_combine(D, d_dtype, M_cap, N, token_row, weights, T, k, out,
+                              static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? FP8_OK
+               : FP8_ERR_LAUNCH;
+}
+
 FP8FG_API int fp8_get_status(void* stream)
 {
-    return read_and_clear_status(static_cast<cudaStream_t>(stream));
+    const int a = read_and_clear_status(static_cast<cudaStream_t>(stream));
+    const int b = read_and_clear_moe_status();
+    return a != FP8_OK ? a : b;
 }
 
 FP8FG_API const char* fp8_status_string(int code)

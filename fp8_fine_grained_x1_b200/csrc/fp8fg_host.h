@@ -27,6 +27,18 @@ int launch_blockscaled_gemm(const uint8_t* A, const float* sA, const uint8_t* B,
 
 cudaError_t launch_selftest_wait(cudaStream_t st);
 
+// MoE dispatch / combine (moe.cu).
+int64_t moe_dispatch_workspace_ints(int64_t P, int G);
+cudaError_t launch_moe_dispatch(const uint8_t* q, const float* sA, int64_t T, int64_t K,
+                                const int32_t* topk, int k, int G, uint8_t* q_out, float* sA_out,
+                                int64_t M_cap, int32_t* offsets, int32_t* token_row,
+                                int32_t* row_token, int32_t* ws, cudaStream_t st);
+cudaError_t launch_moe_combine(const void* D, int d_dtype, int64_t M_cap, int64_t N,
+                               const int32_t* token_row, const float* w, int64_t T, int k, void* out,
+                               cudaStream_t st);
+// Read and clear the dispatch kernels' error word (caller synchronised).
+int read_and_clear_moe_status();
+
 // Synchronise `st`, then read and clear the current device's status word.
 int read_and_clear_status(cudaStream_t st);
 

@@ -1,0 +1,253 @@
+// moe.cu -- FP8 dispatch of MoE activations into expert-contiguous groups and
+// the weighted combine of the expert outputs (sm_100a).
+//
+// The recipe caches and dispatches MoE activations in FP8 ("5 Ways You can
+// get More Deepseek While Spending Less" and the cameseeing.com post: cache
+// and dispatch activations in FP8; "Three Fast Methods To Study Deepseek":
+// 8 routed experts per token; gnrental.net post: the MoE part loads the
+// parameters of one expert per group).  Tokens are quantized once (1x128,
+// row-local), and their E4M3 rows and scales -- not BF16 rows -- are moved to
+// the layout the grouped GEMM reads.
+//
+// Dispatch is a stable counting sort of the (token, slot) pairs by expert:
+//   k_moe_count   per chunk of 1024 pairs: expert histogram -> workspace
+//   k_moe_scan    per expert: exclusive prefix over chunks; padded group
+//                 offsets (multiples of 128) -> workspace bases, offsets[]
+//   k_moe_rank    per chunk, one warp in pair order: stable rank of each pair
+//                 among equal experts (__match_any_sync) -> token_row[],
+//                 row_token[]
+//   k_moe_rows    per destination row: copy the token's codes (or zeros for
+//                 padding) and its 1x128 scales (or 1 for padding)
+// Padding rows get codes 0 and scale 1: exactly what quantizing a zero row
+// gives, so the result equals quantizing the gathered BF16 rows.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "fp8fg_device.cuh"
+#include "fp8fg_host.h"
+
+namespace fp8fg {
+
+namespace {
+
+constexpr int kPairsPerChunk = 1024;
+
+// Records a malformed routing entry / capacity overflow (first error wins).
+__device__ int g_moe_status = 0;
+
+__global__ void __launch_bounds__(256) k_moe_count(const int32_t* __restrict__ topk, int64_t P,
+                                                   int G, int32_t* __restrict__ ws)
+{
+    extern __shared__ int32_t hist[];
+    for (int e = threadIdx.x; e < G; e += blockDim.x) hist[e] = 0;
+    __syncthreads();
+    const int64_t i0 = (int64_t)blockIdx.x * kPairsPerChunk;
+    for (int i = threadIdx.x; i < kPairsPerChunk; i += blockDim.x) {
+        const int64_t idx = i0 + i;
+        if (idx >= P) break;
+        const int32_t e = topk[idx];
+        if (e >= 0 && e < G) atomicAdd(&hist[e], 1);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < G; e += blockDim.x) ws[(int64_t)blockIdx.x * G + e] = hist[e];
+}
+
+// One CTA; thread e walks the chunks of expert e.  ws[c][e] becomes the first
+// destination row of expert e's pairs in chunk c.
+__global__ void __launch_bounds__(1024) k_moe_scan(int32_t* __restrict__ ws, int nchunks, int G,
+                                                   int64_t M_cap, int32_t* __restrict__ offsets)
+{
+    __shared__ int32_t padded[1024];
+    __shared__ int32_t base[1025];
+    const int e = threadIdx.x;
+    int32_t total = 0;
+    if (e < G) {
+        for (int c = 0; c < nchunks; ++c) {
+            const int32_t v = ws[(int64_t)c * G + e];
+            ws[(int64_t)c * G + e] = total;
+            total += v;
+        }
+        padded[e] = (total + 127) / 128 * 128;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int64_t acc = 0;
+        for (int j = 0; j < G; ++j) {
+            base[j] = (int32_t)acc;
+            acc += padded[j];
+        }
+        base[G] = (int32_t)(acc < 0x7FFFFFFF ? acc : 0x7FFFFFFF);
+        if (acc > M_cap) atomicCAS(&g_moe_status, 0, FP8_ERR_SHAPE);
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j <= G; j += blockDim.x) offsets[j] = base[j];
+    if (e < G)
+        for (int c = 0; c < nchunks; ++c) ws[(int64_t)c * G + e] += base[e];
+}
+
+// One warp per chunk walks its pairs in order, 32 at a time.
+__global__ void __launch_bounds__(32) k_moe_rank(const int32_t* __restrict__ topk, int64_t P, int k,
+                                                 int G, const int32_t* __restrict__ ws,
+                                                 int64_t M_cap, int32_t* __restrict__ token_row,
+                                                 int32_t* __restrict__ row_token)
+{
+    extern __shared__ int32_t cursor[];
+    const int lane = threadIdx.x;
+    for (int e = lane; e < G; e += 32) cursor[e] = ws[(int64_t)blockIdx.x * G + e];
+    __syncwarp();
+    const int64_t i0 = (int64_t)blockIdx.x * kPairsPerChunk;
+    for (int s = 0; s < kPairsPerChunk; s += 32) {
+        const int64_t idx = i0 + s + lane;
+        const bool live = idx < P;
+        int32_t e = live ? topk[idx] : -1;
+        const bool ok = live && e >= 0 && e < G;
+        if (live && !ok) atomicCAS(&g_moe_status, 0, FP8_ERR_SHAPE);
+        if (!ok) e = -1 - lane;                 // unique key: never matches another lane
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        const unsigned below = same & ((1u << lane) - 1u);
+        int32_t pos = -1;
+        if (ok) pos = cursor[e] + __popc(below);
+        __syncwarp();
+        if (ok && below == 0) cursor[e] += __popc(same);   // lowest lane of the group advances
+        __syncwarp();
+        if (live) {
+            const bool fits = ok && pos >= 0 && pos < M_cap;
+            if (ok && !fits) atomicCAS(&g_moe_status, 0, FP8_ERR_SHAPE);
+            token_row[idx] = fits ? pos : -1;
+            if (fits) row_token[pos] = (int32_t)(idx / k);
+        }
+    }
+}
+
+// CTA = 8 warps, one destination row per warp: the row's K code bytes in
+// 16-byte vectors, then its K/128 scales.
+__global__ void __launch_bounds__(256) k_moe_rows(const uint8_t* __restrict__ q,
+                                                  const float* __restrict__ sA, int64_t T, int64_t K,
+                                                  const int32_t* __restrict__ row_token,
+                                                  int64_t M_cap, uint8_t* __restrict__ q_out,
+                                                  float* __restrict__ sA_out)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (r >= M_cap) return;
+    const int32_t t = row_token[r];
+    uint4* dst = reinterpret_cast<uint4*>(q_out + r * K);
+    const int64_t nvec = K / 16;
+    if (t >= 0 && t < T) {
+        const uint4* src = reinterpret_cast<const uint4*>(q + (int64_t)t * K);
+        for (int64_t v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
+        for (int64_t kb = lane; kb < K / 128; kb += 32) sA_out[kb * M_cap + r] = __ldg(sA + kb * T + t);
+    } else {
+        for (int64_t v = lane; v < nvec; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
+        for (int64_t kb = lane; kb < K / 128; kb += 32) sA_out[kb * M_cap + r] = 1.0f;
+    }
+}
+
+// out[t][:] = sum_j w[t][j] * D[token_row[t][j]][:], FP32 sums, BF16 out.
+// CTA = 256 threads per token row of N columns (8 columns per thread step).
+// Entries of token_row outside [0, M_cap) are skipped like dropped pairs.
+template <typename Tin>
+__global__ void __launch_bounds__(256) k_moe_combine(const Tin* __restrict__ D, int64_t M_cap,
+                                                     int64_t N,
+                                                     const int32_t* __restrict__ token_row,
+                                                     const float* __restrict__ w, int k,
+                                                     __nv_bfloat16* __restrict__ out)
+{
+    const int64_t t = blockIdx.x;
+    for (int64_t c = (int64_t)threadIdx.x * 8; c < N; c += 256 * 8) {
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int j = 0; j < k; ++j) {
+            const int32_t r = token_row[t * k + j];
+            if (r < 0 || r >= M_cap) continue;
+            const float wj = w[t * k + j];
+            if constexpr (sizeof(Tin) == 2) {
+                const uint4 v = __ldg(reinterpret_cast<const uint4*>(D + (int64_t)r * N + c));
+                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    acc[2 * i] = fmaf(wj, __uint_as_float(u[i] << 16), acc[2 * i]);
+                    acc[2 * i + 1] = fmaf(wj, __uint_as_float(u[i] & 0xFFFF0000u), acc[2 * i + 1]);
+                }
+            } else {
+                const float4 a = __ldg(reinterpret_cast<const float4*>(D + (int64_t)r * N + c));
+                const float4 b = __ldg(reinterpret_cast<const float4*>(D + (int64_t)r * N + c) + 1);
+                const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = fmaf(wj, f[i], acc[i]);
+            }
+        }
+        uint4 o;
+        __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[0], acc[1]);
+        __nv_bfloat162 h1 = __floats2bfloat162_rn(acc[2], acc[3]);
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[4], acc[5]);
+        __nv_bfloat162 h3 = __floats2bfloat162_rn(acc[6], acc[7]);
+        o.x = *reinterpret_cast<uint32_t*>(&h0);
+        o.y = *reinterpret_cast<uint32_t*>(&h1);
+        o.z = *reinterpret_cast<uint32_t*>(&h2);
+        o.w = *reinterpret_cast<uint32_t*>(&h3);
+        *reinterpret_cast<uint4*>(out + t * N + c) = o;
+    }
+}
+
+}  // namespace
+
+int64_t moe_dispatch_workspace_ints(int64_t P, int G)
+{
+    return ((P + kPairsPerChunk - 1) / kPairsPerChunk) * (int64_t)G;
+}
+
+cudaError_t launch_moe_dispatch(const uint8_t* q, const float* sA, int64_t T, int64_t K,
+                                const int32_t* topk, int k, int G, uint8_t* q_out, float* sA_out,
+                                int64_t M_cap, int32_t* offsets, int32_t* token_row,
+                                int32_t* row_token, int32_t* ws, cudaStream_t st)
+{
+    const int64_t P = T * k;
+    const int nchunks = (int)((P + kPairsPerChunk - 1) / kPairsPerChunk);
+    // rows beyond the real ones are padding until the rank pass claims them
+    cudaError_t err = cudaMemsetAsync(row_token, 0xFF, (size_t)M_cap * sizeof(int32_t), st);
+    if (err != cudaSuccess) return err;
+    if (nchunks > 0) {
+        k_moe_count<<<nchunks, 256, G * sizeof(int32_t), st>>>(topk, P, G, ws);
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
+    k_moe_scan<<<1, 1024, 0, st>>>(ws, nchunks, G, M_cap, offsets);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (nchunks > 0) {
+        k_moe_rank<<<nchunks, 32, G * sizeof(int32_t), st>>>(topk, P, k, G, ws, M_cap, token_row,
+                                                            row_token);
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
+    if (M_cap > 0)
+        k_moe_rows<<<(unsigned)((M_cap + 7) / 8), 256, 0, st>>>(q, sA, T, K, row_token, M_cap,
+                                                              q_out, sA_out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_moe_combine(const void* D, int d_dtype, int64_t M_cap, int64_t N,
+                               const int32_t* token_row, const float* w, int64_t T, int k, void* out,
+                               cudaStream_t st)
+{
+    if (T == 0) return cudaSuccess;
+    if (d_dtype == FP8_OUT_BF16)
+        k_moe_combine<__nv_bfloat16><<<(unsigned)T, 256, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(D), M_cap, N, token_row, w, k,
+            static_cast<__nv_bfloat16*>(out));
+    else
+        k_moe_combine<float><<<(unsigned)T, 256, 0, st>>>(static_cast<const float*>(D), M_cap, N,
+                                                          token_row, w, k,
+                                                          static_cast<__nv_bfloat16*>(out));
+    return cudaGetLastError();
+}
+
+int read_and_clear_moe_status()
+{
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_moe_status, sizeof(int)) != cudaSuccess) return FP8_ERR_DEVICE;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_moe_status, &zero, sizeof(int)) != cudaSuccess) return FP8_ERR_DEVICE;
+    return v;
+}
+
+}  // namespace fp8fg

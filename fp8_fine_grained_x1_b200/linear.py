@@ -10,8 +10,8 @@ called, issues only library calls on the current stream:
                orientation); dX[M,K_in] = dY . W, W read MN-major
   WgradStep    X[T,C_in], dY[T,C_out] --128x1--> token-contiguous codes with
                per-channel scales; dW[C_out,C_in] = dY^T . X, FP32 out
-  MoeStep      expert-ordered rows A[M_total,K] --1x128-->; W[G,N,K]
-               --128x128-->; grouped GEMM per expert
+  MoeStep      tokens X[T,K] --1x128-->, FP8 dispatch of the rows to
+               expert-contiguous groups; W[G,N,K] --128x128-->; grouped GEMM
 
 ("5 Ways You can get More Deepseek While Spending Less", Figure 6: Fprop,
 Dgrad and Wgrad all run in FP8; why-be.co.kr / cameseeing.com posts and
@@ -25,7 +25,8 @@ from __future__ import annotations
 import torch
 
 from . import (B_KMAJOR, B_MNMAJOR, SCALE_FP32, fp8_blockscaled_gemm, fp8_grouped_gemm,
-               fp8_quant_act_128x1, fp8_quant_act_1x128, fp8_quant_w_128x128)
+               fp8_moe_combine, fp8_moe_dispatch, fp8_moe_dispatch_workspace_bytes,
+               fp8_quant_act_128x1, fp8_quant_act_1x128, fp8_quant_w_128x128, moe_capacity)
 
 
 def _empty(shape, dtype, device):
@@ -119,28 +120,50 @@ class WgradStep:
 
 
 class MoeStep:
-    kernel_calls = 3
+    """MoE expert layer forward: tokens X[T,K] --1x128--> FP8 rows, FP8
+    dispatch to expert-contiguous 128-padded groups (fp8_moe_dispatch),
+    W[G,N,K] --128x128-->, grouped GEMM.  `combine(weights)` adds the
+    weighted return to token order."""
+    kernel_calls = 7      # quantize X, 4 dispatch kernels, quantize W, grouped GEMM (+1 memset)
 
-    def __init__(self, a, w, offsets, out_dtype=torch.bfloat16, scale_mode=SCALE_FP32):
-        M_total, K = a.shape
+    def __init__(self, x, topk, w, out_dtype=torch.bfloat16, scale_mode=SCALE_FP32):
+        T, K = x.shape
         G, N, K2 = w.shape
         assert K == K2
-        d = a.device
-        self.a, self.w, self.offsets, self.mode = a, w, offsets, scale_mode
-        self.qa = _empty((M_total, K), torch.uint8, d)
-        self.sa = _empty((K // 128, M_total), torch.float32, d)
+        k = topk.shape[1]
+        d = x.device
+        self.x, self.topk, self.w, self.mode, self.G = x, topk, w, scale_mode, G
+        self.qx = _empty((T, K), torch.uint8, d)
+        self.sx = _empty((K // 128, T), torch.float32, d)
+        self.M_cap = moe_capacity(T, k, G)
+        self.qa = _empty((self.M_cap, K), torch.uint8, d)
+        self.sa = _empty((K // 128, self.M_cap), torch.float32, d)
+        self.offsets = _empty((G + 1,), torch.int32, d)
+        self.token_row = _empty((T, k), torch.int32, d)
+        self.row_token = _empty((self.M_cap,), torch.int32, d)
+        self.ws = _empty((max(1, fp8_moe_dispatch_workspace_bytes(T, k, G) // 4),), torch.int32, d)
         self.qw = _empty((G, N, K), torch.uint8, d)
         self.sw = _empty((G, N // 128, K // 128), torch.float32, d)
-        self.y = _empty((M_total, N), out_dtype, d)
+        self.y = _empty((self.M_cap, N), out_dtype, d)
+        self.out = None
 
     def quantize(self, stream=None):
-        fp8_quant_act_1x128(self.a, self.qa, self.sa, self.mode, stream)
+        fp8_quant_act_1x128(self.x, self.qx, self.sx, self.mode, stream)
+        fp8_moe_dispatch(self.qx, self.sx, self.topk, self.G, self.qa, self.sa, self.offsets,
+                         self.token_row, self.row_token, self.ws, stream)
         G, N, K = self.w.shape
         fp8_quant_w_128x128(self.w.view(G * N, K), self.qw.view(G * N, K),
                             self.sw.view(G * N // 128, K // 128), self.mode, stream)
 
     def gemm(self, stream=None):
         fp8_grouped_gemm(self.qa, self.sa, self.qw, self.sw, self.offsets, self.y, stream)
+
+    def combine(self, weights, stream=None):
+        T = self.x.shape[0]
+        if self.out is None:
+            self.out = _empty((T, self.y.shape[1]), torch.bfloat16, self.x.device)
+        fp8_moe_combine(self.y, self.token_row, weights, self.out, stream)
+        return self.out
 
     def __call__(self, stream=None):
         self.quantize(stream)

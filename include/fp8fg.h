@@ -27,8 +27,9 @@
  * Conventions shared by every entry point
  *   - Every tensor pointer is caller-owned DEVICE memory on the current CUDA
  *     device (e.g. PyTorch-allocated).  The library allocates nothing and
- *     keeps no per-call state; its only global state is one status word per
- *     device (a __device__ variable) and a host-side wait time limit.
+ *     keeps no per-call state; its only global state is two status words per
+ *     device (__device__ variables: one for the GEMM, one for the MoE
+ *     dispatch) and a host-side wait time limit.
  *   - All calls are asynchronous on `stream` (a cudaStream_t; NULL is the
  *     legacy default stream).  None synchronises except fp8_get_status().
  *   - Arguments are validated on the host before anything is launched; on a
@@ -169,6 +170,53 @@ int fp8_blockscaled_gemm(const uint8_t* A, const float* sA, const uint8_t* B, in
 int fp8_grouped_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB,
                      const int32_t* group_offsets, int G, int64_t M_total, int64_t N, int64_t K,
                      void* D, int out_dtype, void* stream);
+
+/*
+ * FP8 dispatch of MoE activations ([P1]/[P3] cache and dispatch activations
+ * in FP8; [P4] top-8 routing): rows of 1x128-quantized tokens, with their
+ * scales, are gathered into expert-contiguous groups, each padded with zero
+ * rows to a multiple of 128 -- the A operand of fp8_grouped_gemm.  Pairs
+ * (token t, slot j) are ordered by expert, then by t, then by j (a stable
+ * counting sort), so the layout is deterministic.
+ *   q          [T][K] E4M3 codes of the tokens, sA [K/128][T] FP32 scales
+ *              (as written by fp8_quant_act_1x128)
+ *   topk       [T][k] int32 expert ids in [0, G), device memory
+ *   q_out      [M_cap][K] E4M3, sA_out [K/128][M_cap] FP32: expert-ordered
+ *              rows; padding rows and rows at or beyond group_offsets[G]
+ *              get codes 0 and scale 1 (exactly a quantized zero row)
+ *   group_offsets [G+1] int32: first row of each group, group_offsets[G] =
+ *              padded total (device memory, written)
+ *   token_row  [T][k] int32: destination row of each pair (for the combine)
+ *   row_token  [M_cap] int32: source token of each row, -1 for padding
+ *   workspace  caller-owned device scratch of fp8_moe_dispatch_workspace_bytes
+ *              bytes (per-chunk expert counts); contents on entry ignored
+ * Sizes: T >= 0; K > 0, K % 128 == 0; 1 <= k; 1 <= G <= 1024; T*k <=
+ * 2^31 - 1 - 1024*128 (so every padded row index fits in int32); M_cap >= 0
+ * and M_cap % 128 == 0; q and q_out 16-byte aligned, the rest 4-byte
+ * aligned.  Argument errors return FP8_ERR_SHAPE / NULL / ALIGN before any
+ * launch.  A padded total above M_cap, or an expert id outside
+ * [0, G), is reported as FP8_ERR_SHAPE through the status word; such pairs get
+ * token_row -1 and are not copied.  Launches four kernels and one memset.
+ */
+int64_t fp8_moe_dispatch_workspace_bytes(int64_t T, int k, int G);
+int fp8_moe_dispatch(const uint8_t* q, const float* sA, int64_t T, int64_t K, const int32_t* topk,
+                     int k, int G, uint8_t* q_out, float* sA_out, int64_t M_cap,
+                     int32_t* group_offsets, int32_t* token_row, int32_t* row_token,
+                     void* workspace, int64_t workspace_bytes, void* stream);
+
+/*
+ * Weighted combine of the expert outputs back to token order:
+ *   out[t][n] = BF16( sum_j w[t][j] * D[token_row[t][j]][n] )  (FP32 sums in
+ * slot order; pairs whose token_row is outside [0, M_cap), e.g. -1, are
+ * skipped).
+ *   D          [M_cap][N] BF16 or FP32 (d_dtype FP8_OUT_*), the grouped GEMM
+ *              output; token_row [T][k] int32 from fp8_moe_dispatch;
+ *   weights    [T][k] FP32 gate weights; out [T][N] BF16
+ * Sizes: T >= 0, k >= 1, N > 0 and N % 8 == 0; D and out 16-byte aligned.
+ * All buffers are caller-owned device memory.  One kernel launch.
+ */
+int fp8_moe_combine(const void* D, int d_dtype, int64_t M_cap, int64_t N, const int32_t* token_row,
+                    const float* weights, int64_t T, int k, void* out, void* stream);
 
 /*
  * Synchronise `stream`, then return and clear the current device's status

@@ -30,7 +30,7 @@ FAKE5 = 0x50000
 def _declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:int|void|const char\*)\s+(fp8_\w+)\s*\(", text, re.M)))
+    return sorted(set(re.findall(r"^\s*(?:int64_t|int|void|const char\*)\s+(fp8_\w+)\s*\(", text, re.M)))
 
 
 @pytest.fixture(scope="module")

@@ -14,6 +14,7 @@ import torch
 import fp8_fine_grained_x1_b200 as fg
 import oracle
 from fp8_fine_grained_x1_b200 import linear, synth
+from oracle import moe as omoe
 
 from gpu_util import assert_gemm_close, d2h, dev
 
@@ -103,43 +104,45 @@ def test_wgrad_token_axis_groups(mode):
 def test_moe_grouped_fprop():
     wl = synth.moe()
     lay = wl["layout"]
-    a = synth.gather_rows(wl["x"].to(dev()), lay.row_token)
     G, N, K = wl["w"].shape
-    off = lay.offsets.numpy()
-    step = linear.MoeStep(a, wl["w"].to(dev()), lay.offsets.to(dev()))
+    topk = lay.topk.to(torch.int32)
+    step = linear.MoeStep(wl["x"].to(dev()), topk.to(dev()), wl["w"].to(dev()))
     y = step()
     torch.cuda.synchronize()
     assert fg.fp8_get_status() == fg.FP8_OK
+    # layout: identical to the generator's independent expert ordering
+    off = step.offsets.cpu().numpy()
+    assert np.array_equal(off, lay.offsets.numpy())
+    assert np.array_equal(step.row_token.cpu().numpy()[:lay.m_total], lay.row_token.numpy())
 
-    # weights: every expert, bit-exact
+    # tokens and weights quantized by the oracle, bit-exact
+    qx, sx = oracle.quant_act_1x128(_bits(wl["x"]))
+    assert np.array_equal(step.qx.cpu().numpy(), qx) and np.array_equal(step.sx.cpu().numpy(), sx)
     qw, sw = oracle.quant_w_128x128(_bits(wl["w"].view(G * N, K)))
     assert np.array_equal(step.qw.cpu().numpy().reshape(G * N, K), qw)
     assert np.array_equal(step.sw.cpu().numpy().reshape(G * N // 128, K // 128), sw)
     qw = qw.reshape(G, N, K)
     sw = sw.reshape(G, N // 128, K // 128)
 
-    # sampled rows: group edges (first, last real, last padding) + random rows
+    # dispatched rows: the oracle's dispatch of the oracle's codes, bit-exact
+    od = omoe.moe_dispatch(qx, sx, topk.numpy(), G, step.M_cap)
+    assert np.array_equal(step.qa.cpu().numpy(), od["q"])
+    assert np.array_equal(step.sa.cpu().numpy(), od["sA"])
+
+    # GEMM at the first, last-real and last-padding row of every expert + random rows
     rng = np.random.default_rng(4)
     rows = set(rng.integers(0, lay.m_total, 64).tolist())
     for e in range(G):
         if off[e + 1] > off[e]:
             rows |= {int(off[e]), int(off[e] + lay.counts[e] - 1), int(off[e + 1] - 1)}
     rows = np.array(sorted(rows))
-    tok = lay.row_token[rows]
-    a_rows = synth.gather_rows(wl["x"], tok)                       # CPU, same rows
-    qa_r, sa_r = oracle.quant_act_1x128(_bits(a_rows))
-    assert np.array_equal(step.qa[torch.from_numpy(rows).to(dev())].cpu().numpy(), qa_r)
-    assert np.array_equal(step.sa[:, torch.from_numpy(rows).to(dev())].cpu().numpy(), sa_r)
-
     yh = d2h(y)
     for e in range(G):
-        sel = np.flatnonzero((rows >= off[e]) & (rows < off[e + 1]))
+        sel = rows[(rows >= off[e]) & (rows < off[e + 1])]
         if sel.size == 0:
             continue
         pts = np.array([(i, n) for i in sel for n in range(N)], np.int64)
-        ref, tol = oracle.gemm_points(qa_r, sa_r, qw[e], sw[e], pts)
-        got = yh[rows[pts[:, 0]], pts[:, 1]]
-        assert_gemm_close(got, ref, tol, True, f"moe expert {e}")
-    # padding rows are exactly zero
-    pad = lay.row_token.numpy() < 0
-    assert np.all(yh[pad] == 0.0)
+        ref, tol = oracle.gemm_points(od["q"], od["sA"], qw[e], sw[e], pts)
+        assert_gemm_close(yh[pts[:, 0], pts[:, 1]], ref, tol, True, f"moe expert {e}")
+    pad = step.row_token.cpu().numpy()[:lay.m_total] < 0
+    assert np.all(yh[:lay.m_total][pad] == 0.0)
