@@ -44,6 +44,7 @@ EXPORTED = (
     "fp8_blockscaled_gemm", "fp8_grouped_gemm", "fp8_get_status", "fp8_status_string",
     "fp8_set_wait_timeout_ns", "fp8_selftest_wait_timeout", "fp8_device_supported",
     "fp8_moe_dispatch_workspace_bytes", "fp8_moe_dispatch", "fp8_moe_combine",
+    "fp8_moe_dispatch_noalloc",
 )
 
 
@@ -93,6 +94,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fp8_moe_dispatch.restype = _I
     lib.fp8_moe_combine.argtypes = [_P, _I, _I64, _I64, _P, _P, _I64, _I, _P, _P]
     lib.fp8_moe_combine.restype = _I
+    lib.fp8_moe_dispatch_noalloc.argtypes = [_P, _P, _I64, _I64, _P, _I, _I, _P, _P, _I64, _P,
+                                             _P, _P, _P]
+    lib.fp8_moe_dispatch_noalloc.restype = _I
     _lib = lib
     return lib
 
@@ -200,6 +204,19 @@ def fp8_moe_dispatch(q, sA, topk, G, q_out, sA_out, group_offsets, token_row, ro
         _ptr(q), _ptr(sA), T, K, _ptr(topk), k, G, _ptr(q_out), _ptr(sA_out), M_cap,
         _ptr(group_offsets), _ptr(token_row), _ptr(row_token), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)), "fp8_moe_dispatch")
+
+
+def fp8_moe_dispatch_noalloc(q, sA, topk, G, q_out, sA_out, group_offsets, token_row, row_token,
+                             stream=None) -> None:
+    """fp8_moe_dispatch with the library's fixed device scratch (no workspace
+    argument; nothing allocated).  Overlapping calls on one device race."""
+    T, K = q.shape
+    k = topk.shape[1]
+    M_cap = q_out.shape[0]
+    _check(load_library().fp8_moe_dispatch_noalloc(
+        _ptr(q), _ptr(sA), T, K, _ptr(topk), k, G, _ptr(q_out), _ptr(sA_out), M_cap,
+        _ptr(group_offsets), _ptr(token_row), _ptr(row_token), _stream(stream)),
+        "fp8_moe_dispatch_noalloc")
 
 
 def fp8_moe_combine(D, token_row, weights, out, stream=None) -> None:

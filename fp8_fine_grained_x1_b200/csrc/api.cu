@@ -189,6 +189,24 @@ FP8FG_API int fp8_moe_dispatch(const uint8_t* q, const float* sA, int64_t T, int
                : FP8_ERR_LAUNCH;
 }
 
+static_assert(kMoeStaticWsInts * (int64_t)sizeof(int32_t) == FP8_MOE_NOALLOC_WS_BYTES,
+              "static dispatch scratch and its advertised size disagree");
+static int32_t g_no_device_ws = 0;
+
+FP8FG_API int fp8_moe_dispatch_noalloc(const uint8_t* q, const float* sA, int64_t T, int64_t K,
+                                       const int32_t* topk, int k, int G, uint8_t* q_out,
+                                       float* sA_out, int64_t M_cap, int32_t* group_offsets,
+                                       int32_t* token_row, int32_t* row_token, void* stream)
+{
+    const int64_t need = fp8_moe_dispatch_workspace_bytes(T, k, G);
+    if (need > FP8_MOE_NOALLOC_WS_BYTES) return FP8_ERR_SHAPE;
+    int32_t* ws = &g_no_device_ws;   // never dereferenced: without a device the call
+                                     // below validates the rest, then returns FP8_ERR_DEVICE
+    if (device_is_sm100() && moe_static_workspace(&ws) != cudaSuccess) return FP8_ERR_DEVICE;
+    return fp8_moe_dispatch(q, sA, T, K, topk, k, G, q_out, sA_out, M_cap, group_offsets,
+                            token_row, row_token, ws, FP8_MOE_NOALLOC_WS_BYTES, stream);
+}
+
 FP8FG_API int fp8_moe_combine(const void* D, int d_dtype, int64_t M_cap, int64_t N,
                               const int32_t* token_row, const float* weights, int64_t T, int k,
                               void* out, void* stream)

@@ -36,6 +36,10 @@ cudaError_t launch_moe_dispatch(const uint8_t* q, const float* sA, int64_t T, in
 cudaError_t launch_moe_combine(const void* D, int d_dtype, int64_t M_cap, int64_t N,
                                const int32_t* token_row, const float* w, int64_t T, int k, void* out,
                                cudaStream_t st);
+// Capacity of the fixed device scratch used by fp8_moe_dispatch_noalloc.
+constexpr int64_t kMoeStaticWsInts = 65536;
+// Address of that scratch on the current device (looked up once per device).
+cudaError_t moe_static_workspace(int32_t** ws);
 // Read and clear the dispatch kernels' error word (caller synchronised).
 int read_and_clear_moe_status();
 

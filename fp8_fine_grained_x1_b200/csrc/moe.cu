@@ -24,6 +24,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 
 #include "fp8fg_device.cuh"
 #include "fp8fg_host.h"
@@ -36,6 +37,11 @@ constexpr int kPairsPerChunk = 1024;
 
 // Records a malformed routing entry / capacity overflow (first error wins).
 __device__ int g_moe_status = 0;
+
+// Fixed dispatch scratch for the non-allocating entry point (one per device
+// context).  Every entry a dispatch reads is written earlier in the same
+// dispatch, so it never needs clearing.
+__device__ __align__(256) int32_t g_moe_static_ws[kMoeStaticWsInts];
 
 __global__ void __launch_bounds__(256) k_moe_count(const int32_t* __restrict__ topk, int64_t P,
                                                    int G, int32_t* __restrict__ ws)
@@ -239,6 +245,26 @@ cudaError_t launch_moe_combine(const void* D, int d_dtype, int64_t M_cap, int64_
                                                           token_row, w, k,
                                                           static_cast<__nv_bfloat16*>(out));
     return cudaGetLastError();
+}
+
+cudaError_t moe_static_workspace(int32_t** ws)
+{
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static int32_t* addr[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        err = cudaGetSymbolAddress(&p, g_moe_static_ws);     // for the current device
+        if (err != cudaSuccess) return err;
+        addr[dev] = static_cast<int32_t*>(p);
+    }
+    *ws = addr[dev];
+    return cudaSuccess;
 }
 
 int read_and_clear_moe_status()

@@ -205,6 +205,26 @@ int fp8_moe_dispatch(const uint8_t* q, const float* sA, int64_t T, int64_t K, co
                      void* workspace, int64_t workspace_bytes, void* stream);
 
 /*
+ * fp8_moe_dispatch without a caller workspace: the same dispatch, writing
+ * the same outputs, with its scratch in a fixed device array of
+ * FP8_MOE_NOALLOC_WS_BYTES inside the library (one per device).  The pages
+ * have no counterpart: this is an integration convenience for callers that
+ * must not allocate (e.g. inside a CUDA graph), and it allocates nothing.
+ *   Limit: fp8_moe_dispatch_workspace_bytes(T, k, G) <= FP8_MOE_NOALLOC_WS_BYTES
+ *          (e.g. T*k <= 2^21 pairs at G = 32), else FP8_ERR_SHAPE.
+ *   The first call on each device looks the array up (cudaGetSymbolAddress
+ *   with that device current); make it before any stream capture.
+ *   Calls that overlap on one device (other streams, other threads) share
+ *   the array and race: serialise them.  No clearing is needed between
+ *   calls.  Other arguments, errors and launches as fp8_moe_dispatch.
+ */
+#define FP8_MOE_NOALLOC_WS_BYTES 262144
+int fp8_moe_dispatch_noalloc(const uint8_t* q, const float* sA, int64_t T, int64_t K,
+                             const int32_t* topk, int k, int G, uint8_t* q_out, float* sA_out,
+                             int64_t M_cap, int32_t* group_offsets, int32_t* token_row,
+                             int32_t* row_token, void* stream);
+
+/*
  * Weighted combine of the expert outputs back to token order:
  *   out[t][n] = BF16( sum_j w[t][j] * D[token_row[t][j]][n] )  (FP32 sums in
  * slot order; pairs whose token_row is outside [0, M_cap), e.g. -1, are
