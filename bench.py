@@ -155,41 +155,48 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- workloads
 
-def make_step(workload, device):
+def describe(workload):
+    """CPU side of a workload: (wl, desc, (M, N, K), quant_bytes, host inputs,
+    make) where make(device) builds the device step.  The reference arm uses
+    the same desc, so both arms print the same config."""
     import torch
     from fp8_fine_grained_x1_b200 import SCALE_FP32, SCALE_POW2, linear, synth
     if workload == "fprop":
         wl = synth.fprop()
-        step = linear.FpropStep(wl["x"].to(device), wl["w"].to(device))
         M, K = wl["x"].shape
         N = wl["w"].shape[0]
         desc = dict(workload="fprop dense-MLP X[4096,7168] x W[18432,7168]^T, bf16 in, "
                     "1x128 act / 128x128 weight E4M3, bf16 out", M=M, N=N, K=K)
         inputs = [wl["x"], wl["w"]]
         quant_bytes = (M * K + N * K) * 3 + (M * K // 128) * 4 + (N * K // 16384) * 4
+
+        def make(d):
+            return linear.FpropStep(wl["x"].to(d), wl["w"].to(d))
     elif workload == "pr1":
         wl = synth.pr1()
-        step = linear.FpropStep(wl["x"].to(device), wl["w"].to(device), out_dtype=torch.float32)
         M, K = wl["x"].shape
         N = wl["w"].shape[0]
         desc = dict(workload="pr1 tiny fprop X[128,512] x W[256,512]^T fp32 in, fp32 out",
                     M=M, N=N, K=K)
         inputs = [wl["x"], wl["w"]]
         quant_bytes = (M * K + N * K) * 5
+
+        def make(d):
+            return linear.FpropStep(wl["x"].to(d), wl["w"].to(d), out_dtype=torch.float32)
     elif workload == "dgrad":
         wl = synth.dgrad()
-        step = linear.DgradStep(wl["dy"].to(device), wl["w"].to(device))
-        M, Kg = wl["dy"].shape
+        M, K = wl["dy"].shape
         N = wl["w"].shape[1]
         desc = dict(workload="dgrad dX[4096,2048] = dY[4096,7168] . W[7168,2048] (W read "
-                    "transposed), bf16 out", M=M, N=N, K=Kg)
-        K = Kg
+                    "transposed), bf16 out", M=M, N=N, K=K)
         inputs = [wl["dy"], wl["w"]]
         quant_bytes = (M * K + K * N) * 3 + (M * K // 128) * 4
+
+        def make(d):
+            return linear.DgradStep(wl["dy"].to(d), wl["w"].to(d))
     elif workload in ("wgrad", "wgrad_pow2"):
         wl = synth.wgrad()
         mode = SCALE_POW2 if workload == "wgrad_pow2" else SCALE_FP32
-        step = linear.WgradStep(wl["x"].to(device), wl["dy"].to(device), scale_mode=mode)
         T, C_in = wl["x"].shape
         C_out = wl["dy"].shape[1]
         M, N, K = C_out, C_in, T
@@ -197,11 +204,13 @@ def make_step(workload, device):
                     f"groups, fp32 out, {'pow2' if mode else 'fp32'} scales", M=M, N=N, K=K)
         inputs = [wl["x"], wl["dy"]]
         quant_bytes = (T * C_in + T * C_out) * 3 + (T // 128) * (C_in + C_out) * 4
+
+        def make(d):
+            return linear.WgradStep(wl["x"].to(d), wl["dy"].to(d), scale_mode=mode)
     elif workload == "moe":
         wl = synth.moe()
         lay = wl["layout"]
         topk = lay.topk.to(torch.int32)
-        step = linear.MoeStep(wl["x"].to(device), topk.to(device), wl["w"].to(device))
         G, N, K = wl["w"].shape
         T = wl["x"].shape[0]
         M = int(lay.counts.sum())
@@ -214,51 +223,75 @@ def make_step(workload, device):
         # once per token (1 B) and written per padded row (1 B); weights 3 B
         quant_bytes = (T * K * 3 + T * K // 32 + (T + lay.m_total) * K + lay.m_total * K // 32
                        + G * N * K * 3)
+
+        def make(d):
+            return linear.MoeStep(wl["x"].to(d), topk.to(d), wl["w"].to(d))
     else:
         raise SystemExit(f"unknown workload {workload}")
-    flops = 2 * M * N * K
-    return step, desc, flops, quant_bytes, inputs
+    return wl, desc, (M, N, K), quant_bytes, inputs, make
 
 
 # ---------------------------------------------------------------- oracle (CPU) timing
 
-def oracle_sample(workload, budget_s: float = 20.0):
-    """Time the CPU oracle on a bounded sample of the workload and extrapolate
-    one step: quantizers timed on a row sample, GEMM on sampled outputs."""
-    import numpy as np
+def _bits(t):
     import torch
-    import oracle
     from fp8_fine_grained_x1_b200 import synth
+    return synth.bf16_bits(t) if t.dtype == torch.bfloat16 else t.numpy()
+
+
+def oracle_sample(workload, budget_s: float = 20.0, described=None):
+    """Time the CPU oracle on a bounded sample of the workload and extrapolate
+    one step: each quantizer timed on a row (or token-block) sample, the GEMM
+    on sampled outputs with the workload's K, layout and scale granularity."""
+    import numpy as np
+    import oracle
+    from fp8_fine_grained_x1_b200 import SCALE_POW2
     oracle.build()
-    if workload != "fprop":
-        workload = "fprop"          # the reference arm is quoted on the default workload
-    M, N, K = 4096, 18432, 7168
-    rows = 64
-    x = synth.activations(rows, K, seed=0, outlier_seed=2)
-    w = synth.normal((256, K), 0.006, 1)
-    xb, wb = synth.bf16_bits(x), synth.bf16_bits(w)
-    t0 = time.perf_counter()
-    qx, sx = oracle.quant_act_1x128(xb)
-    qw, sw = oracle.quant_w_128x128(wb)
-    t_quant = time.perf_counter() - t0
-    quant_elems = rows * K + 256 * K
+    wl, desc, (M, N, K), _, _, _ = described or describe(workload)
     rng = np.random.default_rng(0)
-    npts = 256
-    t_gemm, done = 0.0, 0
-    while t_gemm < budget_s * 0.8 and done < 200000:
-        pts = np.stack([rng.integers(0, rows, npts), rng.integers(0, 256, npts)], 1)
+    mode = SCALE_POW2 if workload == "wgrad_pow2" else oracle.SCALE_FP32
+    gemm_kw = {}
+    t0 = time.perf_counter()
+    if workload in ("fprop", "pr1", "dgrad", "moe"):
+        xa = wl["dy"] if workload == "dgrad" else wl["x"]
+        w = wl["w"].reshape(-1, wl["w"].shape[-1])
+        ra, rw = min(64, xa.shape[0]), min(256, w.shape[0])
+        qa, sa = oracle.quant_act_1x128(_bits(xa[:ra]), mode)
+        qb, sb = oracle.quant_w_128x128(_bits(w[:rw]), mode)
+        q_done, q_total = ra * xa.shape[1] + rw * w.shape[1], xa.numel() + w.numel()
+        if workload == "dgrad":
+            # W stored [K][N]: the sample keeps its first 256 K-rows, all N columns
+            gemm_kw = dict(b_major=oracle.B_MNMAJOR)
+            pts_k, m_hi, n_hi = rw, ra, qb.shape[1]
+            qa = np.ascontiguousarray(qa[:, :rw])
+            sa = np.ascontiguousarray(sa[:rw // 128])
+        else:
+            pts_k, m_hi, n_hi = K, ra, rw
+    else:                                            # wgrad: 128x1 along 128 tokens
+        x, dy = wl["x"][:128], wl["dy"][:128]
+        qb, sb = oracle.quant_act_128x1(_bits(x), mode)
+        qa, sa = oracle.quant_act_128x1(_bits(dy), mode)
+        q_done, q_total = x.numel() + dy.numel(), wl["x"].numel() + wl["dy"].numel()
+        gemm_kw = dict(sb_gran=1)
+        pts_k, m_hi, n_hi = 128, qa.shape[0], qb.shape[0]
+    t_quant = time.perf_counter() - t0
+    npts, t_gemm, done = 256, 0.0, 0
+    while t_gemm < budget_s * 0.8 and done < 400000:
+        pts = np.stack([rng.integers(0, m_hi, npts), rng.integers(0, n_hi, npts)], 1)
         t0 = time.perf_counter()
-        oracle.gemm_points(qx, sx, qw, sw, pts)
+        oracle.gemm_points(qa, sa, qb, sb, pts, **gemm_kw)
         t_gemm += time.perf_counter() - t0
         done += npts
         npts = min(npts * 2, 65536)
-    per_point = t_gemm / done
-    per_elem_q = t_quant / quant_elems
-    step_s = per_point * M * N + per_elem_q * (M * K + N * K)
+    # an output's cost grows with K: scale the sampled K to the workload's
+    per_point = t_gemm / done * (K / pts_k)
+    step_s = per_point * M * N + t_quant / q_done * q_total
     flops = 2.0 * M * N * K
-    return dict(value=flops / step_s / 1e12, unit="TFLOP/s", cores=oracle.num_threads(), kind="oracle",
-                sample=f"fprop: 1x128/128x128 quantization of {rows}+256 rows and {done} "
-                       f"GEMM outputs (K=7168, FP64), extrapolated to one 4096x18432x7168 step",
+    return dict(value=flops / step_s / 1e12, unit="TFLOP/s", cores=oracle.num_threads(),
+                kind="oracle",
+                sample=f"{workload}: quantization of {q_done} of {q_total} elements and "
+                       f"{done} GEMM outputs at K={pts_k} (FP64), extrapolated to one "
+                       f"{M}x{N}x{K} step",
                 step_s=step_s)
 
 
@@ -284,22 +317,24 @@ def main():
         if rank != 0:
             return
         t0 = time.perf_counter()
+        described = describe(args.workload)
+        M, N, K = described[2]
         res = None
-        for _ in range(max(1, args.warmup)):
-            pass
         vals = []
         for _ in range(max(1, args.steps)):
-            res = oracle_sample(args.workload, budget_s=max(2.0, 60.0 / max(1, args.steps)))
+            res = oracle_sample(args.workload, budget_s=max(2.0, 60.0 / max(1, args.steps)),
+                                described=described)
             vals.append(res["value"])
         total = time.perf_counter() - t0
         v = sorted(vals)[len(vals) // 2]
         line = {"impl": "reference", "metric": "FP8 block-scaled GEMM TFLOP/s (step incl. "
                 "quantization)", "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
                 "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": res["step_s"] * 1e3, "higher_is_better": True,
+                "ms_per_step": 2.0 * M * N * K / (v * 1e12) * 1e3, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": "fprop dense-MLP X[4096,7168] x W[18432,7168]^T"},
-                "cpu_baseline": {k: res[k] for k in ("value", "unit", "cores", "kind", "sample")},
+                "config": dict(described[1], parallelism="reference arm: CPU oracle, rank 0"),
+                "cpu_baseline": dict({k: res[k] for k in ("unit", "cores", "kind", "sample")},
+                                     value=v),
                 "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0},
                 "wall_s": total}
@@ -319,7 +354,9 @@ def main():
     fg.load_library()
     assert fg.fp8_device_supported(), "needs an sm_100 GPU"
 
-    step, desc, flops, quant_bytes, host_inputs = make_step(args.workload, device)
+    described = describe(args.workload)
+    _, desc, (M_, N_, K_), quant_bytes, host_inputs, make = described
+    step, flops = make(device), 2 * M_ * N_ * K_
     stream = torch.cuda.current_stream()
 
     def barrier():
@@ -410,7 +447,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res = oracle_sample(args.workload)
+        res = oracle_sample(args.workload, described=described)
         cpu = {k: res[k] for k in ("value", "unit", "cores", "kind", "sample")}
 
     if rank == 0:
