@@ -81,6 +81,8 @@ def _load():
     lib.oracle_limited_dot.restype = ctypes.c_double
     lib.oracle_e4m3_encode_array.argtypes = [_P, _I64, _P]
     lib.oracle_e4m3_encode_array.restype = None
+    lib.oracle_requant_1x128_to_128x1.argtypes = [_P, _I64, _P, _I64, _I64, _P, _I64, _P, _I]
+    lib.oracle_requant_1x128_to_128x1.restype = None
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = _I
     _lib = lib
@@ -152,6 +154,20 @@ def quant_act_128x1(x: np.ndarray, mode: int = SCALE_FP32):
     s = np.empty((T // 128, C), np.float32)
     _load().oracle_quant_act_128x1(_ptr(x), dt, T, C, C, _ptr(q), T, _ptr(s), mode)
     return q, s
+
+
+def requant_1x128_to_128x1(q: np.ndarray, sA: np.ndarray, mode: int = SCALE_FP32):
+    """Activations cached as 1x128 FP8 (q [T, C] codes, sA [C/128, T]) regrouped
+    for Wgrad: dequantize to FP32, then 128x1 groups along tokens (reading R13).
+    Returns (qT [C, T] uint8, s [T/128, C] float32)."""
+    q = np.ascontiguousarray(q, np.uint8)
+    sA = np.ascontiguousarray(sA, np.float32)
+    T, C = q.shape
+    assert sA.shape == (C // 128, T) and T % 128 == 0 and C % 128 == 0
+    qT = np.empty((C, T), np.uint8)
+    s = np.empty((T // 128, C), np.float32)
+    _load().oracle_requant_1x128_to_128x1(_ptr(q), C, _ptr(sA), T, C, _ptr(qT), T, _ptr(s), mode)
+    return qT, s
 
 
 def quant_w_128x128(w: np.ndarray, mode: int = SCALE_FP32):

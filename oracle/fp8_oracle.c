@@ -37,6 +37,10 @@
  *       amax <= 448 * 2^e, clamped to e >= -126; codes E(x * 2^-e) exactly.
  *   R5  GEMM reference: sum over K-blocks of sA * sB * P in FP64, with P the
  *       exact FP64 dot product of the decoded E4M3 values inside the block.
+ *   R13 requantizing cached 1x128 FP8 activations for Wgrad: each element is
+ *       dequantized to fl32(decode(q) * sA) (the exact product rounded once
+ *       to FP32), and those FP32 values are quantized in 128x1 groups
+ *       exactly as an FP32 input would be.
  *
  * Every routine is single-purpose and written straight from the definition;
  * OpenMP only splits independent outputs across threads.
@@ -247,6 +251,39 @@ ORACLE_API void oracle_quant_act_128x1(const void* x, int dtype, int64_t T, int6
             out_idx[i] = c * ldqT + tb * 128 + i;
         }
         s[tb * C + c] = quantize_group(x, dtype, in_idx, qT, out_idx, 128, mode);
+    }
+}
+
+/*
+ * Backward-pass requantization of activations cached in FP8 (gnrental.net
+ * post, mixed precision framework: the FP8 Wgrad GEMM lets activations be
+ * stored in FP8 for the backward pass; why-be.co.kr and cameseeing.com
+ * posts: activations are cached in FP8 with the fine-grained grouping).
+ * The cached form is 1x128 (per token, 128 channels); Wgrad wants 128x1
+ * groups along tokens.  Reading R13: dequantize, then group again.
+ *   q   [T][ldq] E4M3 codes of the 1x128 tiles; sA [C/128][T] floats
+ *       (sA[cb*T + t]); codes 0x7F/0xFF (NaN) are outside the domain
+ *   qT  [C][ldqT] bytes, s [T/128][C] floats: as oracle_quant_act_128x1
+ */
+ORACLE_API void oracle_requant_1x128_to_128x1(const uint8_t* q, int64_t ldq, const float* sA,
+                                              int64_t T, int64_t C, uint8_t* qT, int64_t ldqT,
+                                              float* s, int mode)
+{
+    int64_t ntb = T / 128, g;
+#pragma omp parallel for schedule(static)
+    for (g = 0; g < ntb * C; g++) {
+        int64_t tb = g / C, c = g % C, in_idx[128], out_idx[128];
+        float xs[128];
+        int i;
+        for (i = 0; i < 128; i++) {
+            int64_t t = tb * 128 + i;
+            /* decode(q) has 4 significant bits, sA 24: the FP64 product is
+             * exact, so the cast is the single FP32 rounding of R13 */
+            xs[i] = (float)(oracle_e4m3_decode(q[t * ldq + c]) * (double)sA[(c / 128) * T + t]);
+            in_idx[i] = i;
+            out_idx[i] = c * ldqT + t;
+        }
+        s[tb * C + c] = quantize_group(xs, ORACLE_IN_FP32, in_idx, qT, out_idx, 128, mode);
     }
 }
 
