@@ -207,6 +207,24 @@ def describe(workload):
 
         def make(d):
             return linear.WgradStep(wl["x"].to(d), wl["dy"].to(d), scale_mode=mode)
+    elif workload == "wgrad_cached":
+        wl = synth.wgrad()
+        T, C_in = wl["x"].shape
+        C_out = wl["dy"].shape[1]
+        M, N, K = C_out, C_in, T
+        desc = dict(workload="wgrad dW[2048,7168] = dY^T . X over 8192 tokens, X from its "
+                    "cached 1x128 FP8 form requantized to 128x1, dY quantized 128x1, fp32 out",
+                    M=M, N=N, K=K)
+        inputs = None
+        # X: cache read and codes written, 1 + 4/128 B each way; dY: 3 + 4/128 B
+        quant_bytes = T * C_in * 2 + 2 * (T // 128) * C_in * 4 + \
+            T * C_out * 3 + (T // 128) * C_out * 4
+
+        def make(d):
+            import fp8_fine_grained_x1_b200 as fg
+            # the forward pass's cache of X, made once outside the timed region
+            qx, sx = fg.quant_act_1x128(wl["x"].to(d))
+            return linear.WgradCachedStep(qx, sx, wl["dy"].to(d))
     elif workload == "moe":
         wl = synth.moe()
         lay = wl["layout"]
@@ -269,7 +287,13 @@ def oracle_sample(workload, budget_s: float = 20.0, described=None):
             pts_k, m_hi, n_hi = K, ra, rw
     else:                                            # wgrad: 128x1 along 128 tokens
         x, dy = wl["x"][:128], wl["dy"][:128]
-        qb, sb = oracle.quant_act_128x1(_bits(x), mode)
+        if workload == "wgrad_cached":
+            t_cache = time.perf_counter()
+            cq, cs = oracle.quant_act_1x128(_bits(x), mode)     # the forward's cache: untimed
+            t0 += time.perf_counter() - t_cache
+            qb, sb = oracle.requant_1x128_to_128x1(cq, cs, mode)
+        else:
+            qb, sb = oracle.quant_act_128x1(_bits(x), mode)
         qa, sa = oracle.quant_act_128x1(_bits(dy), mode)
         q_done, q_total = x.numel() + dy.numel(), wl["x"].numel() + wl["dy"].numel()
         gemm_kw = dict(sb_gran=1)
@@ -303,7 +327,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="fprop",
-                    choices=["fprop", "pr1", "dgrad", "wgrad", "wgrad_pow2", "moe"])
+                    choices=["fprop", "pr1", "dgrad", "wgrad", "wgrad_pow2", "wgrad_cached",
+                             "moe"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -357,6 +382,8 @@ def main():
     described = describe(args.workload)
     _, desc, (M_, N_, K_), quant_bytes, host_inputs, make = described
     step, flops = make(device), 2 * M_ * N_ * K_
+    if host_inputs is None:          # inputs made on the device (e.g. a forward-pass cache)
+        host_inputs = [t.cpu() for t in step.inputs]
     stream = torch.cuda.current_stream()
 
     def barrier():
@@ -416,8 +443,8 @@ def main():
     e2e = None
     if args.e2e_steps > 0:
         pinned = [t.contiguous().pin_memory() for t in host_inputs]
-        dev_inputs = [step_input for step_input in _step_inputs(step)]
-        out_dev = _step_output(step)
+        dev_inputs = list(step.inputs)
+        out_dev = step.output
         out_host = torch.empty(out_dev.shape, dtype=out_dev.dtype, pin_memory=True)
         h2d = sum(t.numel() * t.element_size() for t in pinned)
         d2h = out_host.numel() * out_host.element_size()
@@ -478,26 +505,6 @@ def main():
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
-
-
-def _step_inputs(step):
-    from fp8_fine_grained_x1_b200 import linear
-    if isinstance(step, linear.FpropStep):
-        return [step.x, step.w]
-    if isinstance(step, linear.DgradStep):
-        return [step.dy, step.w]
-    if isinstance(step, linear.WgradStep):
-        return [step.x, step.dy]
-    return [step.x, step.w, step.topk]
-
-
-def _step_output(step):
-    from fp8_fine_grained_x1_b200 import linear
-    if isinstance(step, linear.DgradStep):
-        return step.dx
-    if isinstance(step, linear.WgradStep):
-        return step.dw
-    return step.y
 
 
 if __name__ == "__main__":

@@ -44,7 +44,7 @@ EXPORTED = (
     "fp8_blockscaled_gemm", "fp8_grouped_gemm", "fp8_get_status", "fp8_status_string",
     "fp8_set_wait_timeout_ns", "fp8_selftest_wait_timeout", "fp8_device_supported",
     "fp8_moe_dispatch_workspace_bytes", "fp8_moe_dispatch", "fp8_moe_combine",
-    "fp8_moe_dispatch_noalloc",
+    "fp8_moe_dispatch_noalloc", "fp8_requant_1x128_to_128x1",
 )
 
 
@@ -97,6 +97,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fp8_moe_dispatch_noalloc.argtypes = [_P, _P, _I64, _I64, _P, _I, _I, _P, _P, _I64, _P,
                                              _P, _P, _P]
     lib.fp8_moe_dispatch_noalloc.restype = _I
+    lib.fp8_requant_1x128_to_128x1.argtypes = [_P, _I64, _P, _I64, _I64, _P, _I64, _P, _I, _P]
+    lib.fp8_requant_1x128_to_128x1.restype = _I
     _lib = lib
     return lib
 
@@ -160,6 +162,15 @@ def fp8_quant_act_128x1(x, qT, s, scale_mode: int = SCALE_FP32, stream=None) -> 
     _check(load_library().fp8_quant_act_128x1(
         _ptr(x), _in_dtype(x), T, C, _row_stride(x), _ptr(qT), _row_stride(qT), _ptr(s),
         scale_mode, _stream(stream)), "fp8_quant_act_128x1")
+
+
+def fp8_requant_1x128_to_128x1(q, sA, qT, s, scale_mode: int = SCALE_FP32, stream=None) -> None:
+    """Cached 1x128 codes q [T, C] with sA [C/128, T] -> dequantize -> qT [C, T],
+    s [T/128, C] in 128x1 groups along tokens."""
+    T, C = q.shape
+    _check(load_library().fp8_requant_1x128_to_128x1(
+        _ptr(q), _row_stride(q), _ptr(sA), T, C, _ptr(qT), _row_stride(qT), _ptr(s),
+        scale_mode, _stream(stream)), "fp8_requant_1x128_to_128x1")
 
 
 def fp8_quant_w_128x128(w, q, sW, scale_mode: int = SCALE_FP32, stream=None) -> None:
@@ -263,6 +274,15 @@ def quant_act_128x1(x, scale_mode: int = SCALE_FP32, stream=None):
     s = torch.empty((T // 128, C), dtype=torch.float32, device=x.device)
     fp8_quant_act_128x1(x, q, s, scale_mode, stream)
     return q, s
+
+
+def requant_1x128_to_128x1(q, sA, scale_mode: int = SCALE_FP32, stream=None):
+    import torch
+    T, C = q.shape
+    qT = torch.empty((C, T), dtype=torch.uint8, device=q.device)
+    s = torch.empty((T // 128, C), dtype=torch.float32, device=q.device)
+    fp8_requant_1x128_to_128x1(q, sA, qT, s, scale_mode, stream)
+    return qT, s
 
 
 def quant_w_128x128(w, scale_mode: int = SCALE_FP32, stream=None):

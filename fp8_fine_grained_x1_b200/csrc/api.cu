@@ -99,6 +99,26 @@ FP8FG_API int fp8_quant_act_128x1(const void* x, int in_dtype, int64_t T, int64_
                : FP8_ERR_LAUNCH;
 }
 
+FP8FG_API int fp8_requant_1x128_to_128x1(const uint8_t* q, int64_t ldq, const float* sA,
+                                         int64_t T, int64_t C, uint8_t* qT, int64_t ldqT,
+                                         float* s, int scale_mode, void* stream)
+{
+    if (!is_mode(scale_mode)) return FP8_ERR_DTYPE;
+    if (T <= 0 || T > kMaxDim || T % 128 || T / 128 > 65535 || C < 0 || C > kMaxDim || C % 128 ||
+        ldq < C || ldqT < T || ldq > kMaxDim || ldqT > kMaxDim)
+        return FP8_ERR_SHAPE;
+    if (C == 0) return FP8_OK;
+    if (!q || !sA || !qT || !s) return FP8_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(qT, 16) || !aligned(sA, 4) || !aligned(s, 4) || ldq % 16 ||
+        ldqT % 16)
+        return FP8_ERR_ALIGN;
+    if (!device_is_sm100()) return FP8_ERR_DEVICE;
+    return launch_requant_128x1(q, ldq, sA, T, C, qT, ldqT, s, scale_mode,
+                                static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? FP8_OK
+               : FP8_ERR_LAUNCH;
+}
+
 FP8FG_API int fp8_quant_w_128x128(const void* w, int in_dtype, int64_t N, int64_t K, int64_t ldw,
                                   uint8_t* q, int64_t ldq, float* sW, int scale_mode, void* stream)
 {

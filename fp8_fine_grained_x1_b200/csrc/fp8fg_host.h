@@ -13,6 +13,9 @@ cudaError_t launch_quant_act_1x128(const void* x, int in_dtype, int64_t M, int64
                                    uint8_t* q, int64_t ldq, float* sA, int mode, cudaStream_t st);
 cudaError_t launch_quant_act_128x1(const void* x, int in_dtype, int64_t T, int64_t C, int64_t ldx,
                                    uint8_t* qT, int64_t ldqT, float* s, int mode, cudaStream_t st);
+cudaError_t launch_requant_128x1(const uint8_t* q, int64_t ldq, const float* sA, int64_t T,
+                                 int64_t C, uint8_t* qT, int64_t ldqT, float* s, int mode,
+                                 cudaStream_t st);
 cudaError_t launch_quant_w_128x128(const void* w, int in_dtype, int64_t N, int64_t K, int64_t ldw,
                                    uint8_t* q, int64_t ldq, float* sW, int mode, cudaStream_t st);
 

@@ -7,11 +7,13 @@
 //   k_quant_1x128    one scale per token per 128 channels
 //   k_quant_128x1    one scale per channel per 128 tokens, written transposed
 //   k_quant_w128     one scale per 128x128 weight block
+//   k_requant_128x1  cached 1x128 codes -> dequantize -> 128x1 groups (Wgrad)
 // Each reads its input once with 16-byte vector loads, reduces the group's
 // max-abs with warp shuffles (plus shared memory for the wider groups),
 // derives the scale with correctly rounded FP32 division, and writes packed
 // E4M3 codes (cvt.rn.satfinite.e4m3x2) with 8- or 16-byte stores.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
@@ -368,6 +370,126 @@ __global__ void __launch_bounds__(kThr128x1, 6) k_quant_128x1(const Tin* __restr
     }
 }
 
+// ------------------------------------------------------------ requantize 1x128 -> 128x1
+
+// Activations cached as 1x128 E4M3 tiles (the forward pass's quantized X)
+// regrouped for the Wgrad GEMM: every code is dequantized to
+// fl32(decode(q) * sA) -- E4M3 -> FP16 -> FP32 is exact, so __fmul_rn gives
+// that single rounding -- and the FP32 values are quantized in 128x1 groups
+// along tokens, exactly as k_quant_128x1 quantizes an FP32 input.
+//
+// CTA = 256 threads per tile of 128 tokens x 128 channels (one channel block,
+// hence one cached scale per token).  The 16 KB code tile is staged with
+// cp.async; warp w then owns tokens 16w .. 16w+15 and lane l channels
+// 4l .. 4l+3, read as one 32-bit word per token (a warp reads a whole
+// 128-byte row, conflict-free).  Pass 1: max-abs, combined over the 8 warps
+// through shared memory.  Pass 2: each thread encodes its 16 tokens of each
+// of its 4 channels into one 16-byte word.  The staged tile is dead by then,
+// so the transposed codes go back into the same shared memory (16-byte chunks
+// XOR-swizzled by (channel / 4) % 8, conflict-free) and leave as coalesced
+// 128-byte rows of qT.
+// Grid: x = C/128, y = T/128.
+constexpr int kReqTok = 128;
+constexpr int kReqCh = 128;
+
+__device__ __forceinline__ void decode4_e4m3(uint32_t w, float (&f)[4])
+{
+    const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xFFFFu), __NV_E4M3);
+    const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w >> 16), __NV_E4M3);
+    const float2 a = __half22float2(__half2(lo));
+    const float2 b = __half22float2(__half2(hi));
+    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+}
+
+__global__ void __launch_bounds__(256) k_requant_128x1(const uint8_t* __restrict__ q, int64_t ldq,
+                                                       const float* __restrict__ sA, int64_t T,
+                                                       int64_t C, uint8_t* __restrict__ qT,
+                                                       int64_t ldqT, float* __restrict__ s, int mode)
+{
+    __shared__ __align__(16) uint8_t tile[kReqTok * kReqCh];      // codes, then transposed codes
+    __shared__ __align__(16) float part[8][kReqCh];
+    __shared__ float scl[kReqTok];
+
+    const int64_t tb = blockIdx.y;
+    const int64_t cb = blockIdx.x;
+    const int64_t t0 = tb * kReqTok;
+    const int64_t c0 = cb * kReqCh;
+    const int w = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int id = threadIdx.x + 256 * i;
+        const int r = id >> 3, j = id & 7;
+        cp_async16(&tile[r * kReqCh + j * 16], q + (t0 + r) * ldq + c0 + j * 16);
+    }
+    if (threadIdx.x < kReqTok) scl[threadIdx.x] = __ldg(sA + cb * T + t0 + threadIdx.x);
+    cp_async_wait_all();
+    __syncthreads();
+
+    // pass 1: max-abs of the dequantized values of channels 4l..4l+3
+    const uint32_t* tw = reinterpret_cast<const uint32_t*>(tile);
+    float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int i = 0; i < 16; ++i) {
+        const int t = w * 16 + i;
+        float f[4];
+        decode4_e4m3(tw[t * (kReqCh / 4) + lane], f);
+        const float sc = scl[t];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) a[j] = fmaxf(a[j], fabsf(__fmul_rn(f[j], sc)));
+    }
+    *reinterpret_cast<float4*>(&part[w][4 * lane]) = make_float4(a[0], a[1], a[2], a[3]);
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const float4 p = *reinterpret_cast<const float4*>(&part[k][4 * lane]);
+        a[0] = fmaxf(a[0], p.x); a[1] = fmaxf(a[1], p.y);
+        a[2] = fmaxf(a[2], p.z); a[3] = fmaxf(a[3], p.w);
+    }
+    GroupScale g[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) g[j] = group_scale(a[j], mode);
+
+    // pass 2: encode 16 tokens x 4 channels into four 16-byte words
+    uint32_t out[4][4];
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+        float v[4][4];   // [token][channel]
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int t = w * 16 + q4 * 4 + u;
+            float f[4];
+            decode4_e4m3(tw[t * (kReqCh / 4) + lane], f);
+            const float sc = scl[t];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) v[u][j] = __fmul_rn(f[j], sc);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) out[j][q4] = encode4(v[0][j], v[1][j], v[2][j], v[3][j], g[j].inv);
+    }
+    __syncthreads();   // every read of the staged codes is done
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int c = 4 * lane + j;
+        const int chunk = w ^ (lane & 7);
+        *reinterpret_cast<uint4*>(&tile[c * kReqTok + chunk * 16]) =
+            make_uint4(out[j][0], out[j][1], out[j][2], out[j][3]);
+    }
+    if (w == 0) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) s[tb * C + c0 + 4 * lane + j] = g[j].s;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int id = threadIdx.x + 256 * i;
+        const int c = id >> 3, chunk = id & 7;
+        const uint4 v = *reinterpret_cast<const uint4*>(&tile[c * kReqTok + ((chunk ^ ((c >> 2) & 7)) * 16)]);
+        *reinterpret_cast<uint4*>(qT + (c0 + c) * ldqT + t0 + chunk * 16) = v;
+    }
+}
+
 }  // namespace
 
 // ------------------------------------------------------------ launchers
@@ -396,6 +518,15 @@ cudaError_t launch_quant_act_128x1(const void* x, int in_dtype, int64_t T, int64
     else
         k_quant_128x1<float><<<grid, kThr128x1, 0, st>>>(static_cast<const float*>(x), C, ldx, qT,
                                                    ldqT, s, mode);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_requant_128x1(const uint8_t* q, int64_t ldq, const float* sA, int64_t T,
+                                 int64_t C, uint8_t* qT, int64_t ldqT, float* s, int mode,
+                                 cudaStream_t st)
+{
+    const dim3 grid((unsigned)(C / kReqCh), (unsigned)(T / kReqTok));
+    k_requant_128x1<<<grid, 256, 0, st>>>(q, ldq, sA, T, C, qT, ldqT, s, mode);
     return cudaGetLastError();
 }
 

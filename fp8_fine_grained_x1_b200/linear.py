@@ -10,6 +10,8 @@ called, issues only library calls on the current stream:
                orientation); dX[M,K_in] = dY . W, W read MN-major
   WgradStep    X[T,C_in], dY[T,C_out] --128x1--> token-contiguous codes with
                per-channel scales; dW[C_out,C_in] = dY^T . X, FP32 out
+  WgradCachedStep  as WgradStep, with X taken from its cached 1x128 FP8
+               form and requantized into 128x1 groups
   MoeStep      tokens X[T,K] --1x128-->, FP8 dispatch of the rows to
                expert-contiguous groups; W[G,N,K] --128x128-->; grouped GEMM
 
@@ -26,7 +28,8 @@ import torch
 
 from . import (B_KMAJOR, B_MNMAJOR, SCALE_FP32, fp8_blockscaled_gemm, fp8_grouped_gemm,
                fp8_moe_combine, fp8_moe_dispatch, fp8_moe_dispatch_workspace_bytes,
-               fp8_quant_act_128x1, fp8_quant_act_1x128, fp8_quant_w_128x128, moe_capacity)
+               fp8_quant_act_128x1, fp8_quant_act_1x128, fp8_quant_w_128x128,
+               fp8_requant_1x128_to_128x1, moe_capacity)
 
 
 def _empty(shape, dtype, device):
@@ -45,6 +48,7 @@ class FpropStep:
         self.qw, self.sw = _empty((N, K), torch.uint8, d), _empty((N // 128, K // 128), torch.float32, d)
         self.y = _empty((M, N), out_dtype, d)
         self.flops = 2 * M * N * K
+        self.inputs, self.output = [x, w], self.y
 
     def quantize(self, stream=None):
         fp8_quant_act_1x128(self.x, self.qx, self.sx, self.mode, stream)
@@ -74,6 +78,7 @@ class DgradStep:
         self.sw = _empty((N_out // 128, K_in // 128), torch.float32, d)
         self.dx = _empty((M, K_in), out_dtype, d)
         self.flops = 2 * M * K_in * N_out
+        self.inputs, self.output = [dy, w], self.dx
 
     def quantize(self, stream=None):
         fp8_quant_act_1x128(self.dy, self.qdy, self.sdy, self.mode, stream)
@@ -105,6 +110,7 @@ class WgradStep:
         self.sdy = _empty((T // 128, C_out), torch.float32, d)
         self.dw = _empty((C_out, C_in), torch.float32, d)
         self.flops = 2 * C_out * C_in * T
+        self.inputs, self.output = [x, dy], self.dw
 
     def quantize(self, stream=None):
         fp8_quant_act_128x1(self.dy, self.qdyT, self.sdy, self.mode, stream)
@@ -112,6 +118,39 @@ class WgradStep:
 
     def gemm(self, stream=None):
         fp8_blockscaled_gemm(self.qdyT, self.sdy, self.qxT, self.sx, self.dw, B_KMAJOR, 1, stream)
+
+    def __call__(self, stream=None):
+        self.quantize(stream)
+        self.gemm(stream)
+        return self.dw
+
+
+class WgradCachedStep:
+    """Wgrad with X kept from the forward pass as 1x128 FP8 (codes qx [T, C_in],
+    scales sx [C_in/128, T]): the cache is requantized into 128x1 groups along
+    tokens instead of quantizing a BF16 copy of X; dY is quantized 128x1."""
+    kernel_calls = 3
+
+    def __init__(self, qx, sx, dy, scale_mode=SCALE_FP32):
+        T, C_in = qx.shape
+        T2, C_out = dy.shape
+        assert T == T2
+        d = qx.device
+        self.qx, self.sx, self.dy, self.mode = qx, sx, dy, scale_mode
+        self.qxT = _empty((C_in, T), torch.uint8, d)
+        self.sxT = _empty((T // 128, C_in), torch.float32, d)
+        self.qdyT = _empty((C_out, T), torch.uint8, d)
+        self.sdy = _empty((T // 128, C_out), torch.float32, d)
+        self.dw = _empty((C_out, C_in), torch.float32, d)
+        self.flops = 2 * C_out * C_in * T
+        self.inputs, self.output = [qx, sx, dy], self.dw
+
+    def quantize(self, stream=None):
+        fp8_quant_act_128x1(self.dy, self.qdyT, self.sdy, self.mode, stream)
+        fp8_requant_1x128_to_128x1(self.qx, self.sx, self.qxT, self.sxT, self.mode, stream)
+
+    def gemm(self, stream=None):
+        fp8_blockscaled_gemm(self.qdyT, self.sdy, self.qxT, self.sxT, self.dw, B_KMAJOR, 1, stream)
 
     def __call__(self, stream=None):
         self.quantize(stream)
@@ -146,6 +185,7 @@ class MoeStep:
         self.sw = _empty((G, N // 128, K // 128), torch.float32, d)
         self.y = _empty((self.M_cap, N), out_dtype, d)
         self.out = None
+        self.inputs, self.output = [x, w, topk], self.y
 
     def quantize(self, stream=None):
         fp8_quant_act_1x128(self.x, self.qx, self.sx, self.mode, stream)

@@ -114,6 +114,25 @@ int fp8_quant_act_128x1(const void* x, int in_dtype, int64_t T, int64_t C, int64
                         uint8_t* qT, int64_t ldqT, float* s, int scale_mode, void* stream);
 
 /*
+ * Requantization of activations cached in FP8 for the backward pass ([P5]:
+ * the FP8 Wgrad GEMM lets activations be stored in FP8 for backward; [P2]/
+ * [P3]: activations cached and dispatched in FP8 with the fine-grained
+ * grouping).  The cache holds 1x128 tiles (fp8_quant_act_1x128's output);
+ * Wgrad needs 128x1 groups along tokens.  Each code is dequantized to
+ * fl32(decode(q) * sA) -- one FP32 rounding -- and those values are
+ * quantized exactly as fp8_quant_act_128x1 quantizes an FP32 input.
+ *   q    [T][ldq] E4M3 codes, sA [C/128][T] FP32 scales (sA[cb*T + t])
+ *   qT   [C][ldqT] E4M3 codes, s [T/128][C] FP32 scales (as fp8_quant_act_128x1)
+ * Sizes: T > 0, T % 128 == 0, T/128 <= 65535; C >= 0, C % 128 == 0 (C == 0
+ * launches nothing); ldq >= C and ldqT >= T, both multiples of 16; q and qT
+ * 16-byte aligned, sA and s 4-byte aligned.  All buffers are caller-owned
+ * device memory; argument errors return before any launch.  One kernel.
+ */
+int fp8_requant_1x128_to_128x1(const uint8_t* q, int64_t ldq, const float* sA, int64_t T,
+                               int64_t C, uint8_t* qT, int64_t ldqT, float* s, int scale_mode,
+                               void* stream);
+
+/*
  * 128x128 weight blocks: one scale per 128 output x 128 input channels
  * ([P2]/[P3]/[P4] Figure 7 (a)).
  *   w    [N][ldw] input, row-major, BF16 or FP32

@@ -1,4 +1,4 @@
-"""Full-size parity of the five workloads, run exactly as bench.py runs them
+"""Full-size parity of the five workloads (plus Wgrad from cached FP8 X), run exactly as bench.py runs them
 (the step objects of fp8_fine_grained_x1_b200.linear, one GPU, persistent
 GEMM grid), against the CPU oracle on the same seeded inputs.
 
@@ -99,6 +99,26 @@ def test_wgrad_token_axis_groups(mode):
     pts = _points(M, N, 3, rows=_edges(M, 128), cols=_edges(N, 256))
     ref, tol = oracle.gemm_points(qdyT, sdy, qxT, sx, pts, sb_gran=1)
     assert_gemm_close(d2h(dw)[pts[:, 0], pts[:, 1]], ref, tol, False, f"wgrad mode={mode}")
+
+
+def test_wgrad_from_cached_fp8_activations():
+    """Wgrad with X taken from its cached 1x128 FP8 form (the forward's cache
+    is made by the oracle here), requantized to 128x1 on the GPU."""
+    wl = synth.wgrad()
+    cq, cs = oracle.quant_act_1x128(_bits(wl["x"]))
+    step = linear.WgradCachedStep(torch.from_numpy(cq).to(dev()), torch.from_numpy(cs).to(dev()),
+                                  wl["dy"].to(dev()))
+    dw = step()
+    torch.cuda.synchronize()
+    assert fg.fp8_get_status() == fg.FP8_OK
+    qxT, sx = oracle.requant_1x128_to_128x1(cq, cs)
+    qdyT, sdy = oracle.quant_act_128x1(_bits(wl["dy"]))
+    assert np.array_equal(step.qxT.cpu().numpy(), qxT) and np.array_equal(step.sxT.cpu().numpy(), sx)
+    assert np.array_equal(step.qdyT.cpu().numpy(), qdyT) and np.array_equal(step.sdy.cpu().numpy(), sdy)
+    M, N = dw.shape
+    pts = _points(M, N, 5, rows=_edges(M, 128), cols=_edges(N, 256))
+    ref, tol = oracle.gemm_points(qdyT, sdy, qxT, sx, pts, sb_gran=1)
+    assert_gemm_close(d2h(dw)[pts[:, 0], pts[:, 1]], ref, tol, False, "wgrad from cache")
 
 
 def test_moe_grouped_fprop():
