@@ -61,14 +61,23 @@ def measured_peaks():
 
 # ---------------------------------------------------------------- ncu traffic
 
-KERNEL_SOURCES = ("fp8_fine_grained_x1_b200/csrc/gemm.cu",
-                  "fp8_fine_grained_x1_b200/csrc/fp8fg_device.cuh")
+KERNEL_SOURCES = {
+    "k_fp8_gemm": ("fp8_fine_grained_x1_b200/csrc/gemm.cu",
+                   "fp8_fine_grained_x1_b200/csrc/fp8fg_device.cuh"),
+    "k_fp8_gemm_mx": ("fp8_fine_grained_x1_b200/csrc/gemm_mx.cu",
+                      "fp8_fine_grained_x1_b200/csrc/fp8fg_device.cuh"),
+}
 
 
-def kernel_source_hash() -> str:
+def gemm_kernel(workload: str) -> str:
+    """The GEMM kernel a workload's step launches."""
+    return "k_fp8_gemm_mx" if workload.endswith("_tc") else "k_fp8_gemm"
+
+
+def kernel_source_hash(kernel: str = "k_fp8_gemm") -> str:
     import hashlib
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -77,7 +86,8 @@ def kernel_source_hash() -> str:
 def profiled_traffic(workload: str):
     """DRAM bytes (read + write) per GEMM launch from the committed ncu summary
     of this workload, if it was captured from the current kernel sources."""
-    path = os.path.join(ROOT, "profiles", f"k_fp8_gemm_{workload}.md")
+    kernel = gemm_kernel(workload)
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     try:
         fields = {}
         with open(path) as f:
@@ -85,7 +95,7 @@ def profiled_traffic(workload: str):
                 if ":" in line and line.startswith("- "):
                     k, v = line[2:].split(":", 1)
                     fields[k.strip()] = v.strip().strip("`")
-        if fields.get("kernel_source_sha256_16") != kernel_source_hash():
+        if fields.get("kernel_source_sha256_16") != kernel_source_hash(kernel):
             return None
         return float(fields["traffic_bytes_per_launch"])
     except Exception:
@@ -161,16 +171,22 @@ def describe(workload):
     the same desc, so both arms print the same config."""
     import torch
     from fp8_fine_grained_x1_b200 import SCALE_FP32, SCALE_POW2, linear, synth
-    if workload == "fprop":
+    if workload in ("fprop", "fprop_pow2_tc"):
         wl = synth.fprop()
+        tc = workload == "fprop_pow2_tc"
         M, K = wl["x"].shape
         N = wl["w"].shape[0]
         desc = dict(workload="fprop dense-MLP X[4096,7168] x W[18432,7168]^T, bf16 in, "
-                    "1x128 act / 128x128 weight E4M3, bf16 out", M=M, N=N, K=K)
+                    "1x128 act / 128x128 weight E4M3, bf16 out"
+                    + (", pow2 scales applied in the tensor cores (UE8M0 block scaling)"
+                       if tc else ""), M=M, N=N, K=K)
         inputs = [wl["x"], wl["w"]]
         quant_bytes = (M * K + N * K) * 3 + (M * K // 128) * 4 + (N * K // 16384) * 4
 
         def make(d):
+            if tc:
+                return linear.FpropStep(wl["x"].to(d), wl["w"].to(d), scale_mode=SCALE_POW2,
+                                        tensor_core_scaling=True)
             return linear.FpropStep(wl["x"].to(d), wl["w"].to(d))
     elif workload == "pr1":
         wl = synth.pr1()
@@ -194,19 +210,23 @@ def describe(workload):
 
         def make(d):
             return linear.DgradStep(wl["dy"].to(d), wl["w"].to(d))
-    elif workload in ("wgrad", "wgrad_pow2"):
+    elif workload in ("wgrad", "wgrad_pow2", "wgrad_pow2_tc"):
         wl = synth.wgrad()
-        mode = SCALE_POW2 if workload == "wgrad_pow2" else SCALE_FP32
+        mode = SCALE_POW2 if workload.startswith("wgrad_pow2") else SCALE_FP32
+        tc = workload == "wgrad_pow2_tc"
         T, C_in = wl["x"].shape
         C_out = wl["dy"].shape[1]
         M, N, K = C_out, C_in, T
         desc = dict(workload=f"wgrad dW[2048,7168] = dY^T . X over 8192 tokens, 128x1 "
-                    f"groups, fp32 out, {'pow2' if mode else 'fp32'} scales", M=M, N=N, K=K)
+                    f"groups, fp32 out, {'pow2' if mode else 'fp32'} scales"
+                    + (", scaled in the tensor cores (UE8M0 block scaling)" if tc else ""),
+                    M=M, N=N, K=K)
         inputs = [wl["x"], wl["dy"]]
         quant_bytes = (T * C_in + T * C_out) * 3 + (T // 128) * (C_in + C_out) * 4
 
         def make(d):
-            return linear.WgradStep(wl["x"].to(d), wl["dy"].to(d), scale_mode=mode)
+            return linear.WgradStep(wl["x"].to(d), wl["dy"].to(d), scale_mode=mode,
+                                    tensor_core_scaling=tc)
     elif workload == "wgrad_cached":
         wl = synth.wgrad()
         T, C_in = wl["x"].shape
@@ -267,10 +287,10 @@ def oracle_sample(workload, budget_s: float = 20.0, described=None):
     oracle.build()
     wl, desc, (M, N, K), _, _, _ = described or describe(workload)
     rng = np.random.default_rng(0)
-    mode = SCALE_POW2 if workload == "wgrad_pow2" else oracle.SCALE_FP32
+    mode = SCALE_POW2 if "pow2" in workload else oracle.SCALE_FP32
     gemm_kw = {}
     t0 = time.perf_counter()
-    if workload in ("fprop", "pr1", "dgrad", "moe"):
+    if workload in ("fprop", "fprop_pow2_tc", "pr1", "dgrad", "moe"):
         xa = wl["dy"] if workload == "dgrad" else wl["x"]
         w = wl["w"].reshape(-1, wl["w"].shape[-1])
         ra, rw = min(64, xa.shape[0]), min(256, w.shape[0])
@@ -327,8 +347,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="fprop",
-                    choices=["fprop", "pr1", "dgrad", "wgrad", "wgrad_pow2", "wgrad_cached",
-                             "moe"])
+                    choices=["fprop", "fprop_pow2_tc", "pr1", "dgrad", "wgrad", "wgrad_pow2",
+                             "wgrad_pow2_tc", "wgrad_cached", "moe"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -491,7 +511,7 @@ def main():
             "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak,
                          "unit": "TFLOP/s", "frac": gemm_tflops / fp8_peak,
                          "traffic": profiled_traffic(args.workload),
-                         "kernel": "k_fp8_gemm", "peak_source":
+                         "kernel": gemm_kernel(args.workload), "peak_source":
                          f"{peaks['source']} sustained bf16 {peaks['bf16_sustained']} TFLOP/s x 2 "
                          f"(FP8/BF16 nominal); burst-based peak {2 * peaks['bf16']}"},
             "quantizers": {"achieved_gbs": quant_gbs, "peak_gbs": peaks["hbm"],

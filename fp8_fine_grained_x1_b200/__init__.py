@@ -33,6 +33,7 @@ FP8_ERR_DTYPE = 4
 FP8_ERR_LAUNCH = 5
 FP8_ERR_TIMEOUT = 6
 FP8_ERR_DEVICE = 7
+FP8_ERR_VALUE = 8
 
 IN_BF16, IN_FP32 = 0, 1
 OUT_BF16, OUT_FP32 = 0, 1
@@ -44,7 +45,7 @@ EXPORTED = (
     "fp8_blockscaled_gemm", "fp8_grouped_gemm", "fp8_get_status", "fp8_status_string",
     "fp8_set_wait_timeout_ns", "fp8_selftest_wait_timeout", "fp8_device_supported",
     "fp8_moe_dispatch_workspace_bytes", "fp8_moe_dispatch", "fp8_moe_combine",
-    "fp8_moe_dispatch_noalloc", "fp8_requant_1x128_to_128x1",
+    "fp8_moe_dispatch_noalloc", "fp8_requant_1x128_to_128x1", "fp8_blockscaled_gemm_pow2",
 )
 
 
@@ -75,6 +76,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         getattr(lib, name).restype = _I
     lib.fp8_blockscaled_gemm.argtypes = [_P, _P, _P, _I, _P, _I, _I64, _I64, _I64, _P, _I, _I64, _P]
     lib.fp8_blockscaled_gemm.restype = _I
+    lib.fp8_blockscaled_gemm_pow2.argtypes = [_P, _P, _P, _I, _P, _I, _I64, _I64, _I64, _P, _I,
+                                              _I64, _P]
+    lib.fp8_blockscaled_gemm_pow2.restype = _I
     lib.fp8_grouped_gemm.argtypes = [_P, _P, _P, _P, _P, _I, _I64, _I64, _I64, _P, _I, _P]
     lib.fp8_grouped_gemm.restype = _I
     lib.fp8_get_status.argtypes = [_P]
@@ -189,6 +193,17 @@ def fp8_blockscaled_gemm(A, sA, B, sB, D, b_major: int = B_KMAJOR, sb_gran: int 
     _check(load_library().fp8_blockscaled_gemm(
         _ptr(A), _ptr(sA), _ptr(B), b_major, _ptr(sB), sb_gran, M, N, K, _ptr(D),
         _out_dtype(D), _row_stride(D), _stream(stream)), "fp8_blockscaled_gemm")
+
+
+def fp8_blockscaled_gemm_pow2(A, sA, B, sB, D, b_major: int = B_KMAJOR, sb_gran: int = 128,
+                              stream=None) -> None:
+    """fp8_blockscaled_gemm for power-of-two scales, scaled inside the tensor
+    cores (UE8M0 block scaling); a scale that is not 2^e reports FP8_ERR_VALUE."""
+    M, K = A.shape
+    N = B.shape[0] if b_major == B_KMAJOR else B.shape[1]
+    _check(load_library().fp8_blockscaled_gemm_pow2(
+        _ptr(A), _ptr(sA), _ptr(B), b_major, _ptr(sB), sb_gran, M, N, K, _ptr(D),
+        _out_dtype(D), _row_stride(D), _stream(stream)), "fp8_blockscaled_gemm_pow2")
 
 
 def fp8_grouped_gemm(A, sA, B, sB, group_offsets, D, stream=None) -> None:

@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libfp8fg.so")
-SOURCES = ["api.cu", "quant.cu", "gemm.cu", "moe.cu"]
+SOURCES = ["api.cu", "quant.cu", "gemm.cu", "gemm_mx.cu", "moe.cu"]
 HEADERS = ["fp8fg_device.cuh", "fp8fg_host.h"]
 
 NVCC_FLAGS = [

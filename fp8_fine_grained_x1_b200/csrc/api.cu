@@ -159,6 +159,28 @@ FP8FG_API int fp8_blockscaled_gemm(const uint8_t* A, const float* sA, const uint
                                    out_dtype, ldd, static_cast<cudaStream_t>(stream));
 }
 
+FP8FG_API int fp8_blockscaled_gemm_pow2(const uint8_t* A, const float* sA, const uint8_t* B,
+                                        int b_major, const float* sB, int sb_gran, int64_t M,
+                                        int64_t N, int64_t K, void* D, int out_dtype, int64_t ldd,
+                                        void* stream)
+{
+    if (!is_out(out_dtype) || (b_major != FP8_B_KMAJOR && b_major != FP8_B_MNMAJOR) ||
+        (sb_gran != 128 && sb_gran != 1) || (sb_gran == 1 && b_major != FP8_B_KMAJOR))
+        return FP8_ERR_DTYPE;
+    if (M < 0 || M > kMaxDim || N <= 0 || N > kMaxDim || N % 128 || K <= 0 || K > kMaxDim ||
+        K % 128 || ldd < N || ldd > kMaxDim)
+        return FP8_ERR_SHAPE;
+    if (M == 0) return FP8_OK;
+    if (!A || !sA || !B || !sB || !D) return FP8_ERR_NULL;
+    const int osz = out_dtype == FP8_OUT_BF16 ? 2 : 4;
+    if (!aligned(A, 16) || !aligned(B, 16) || !aligned(D, 16) || !aligned(sA, 4) ||
+        !aligned(sB, 4) || (ldd * osz) % 16)
+        return FP8_ERR_ALIGN;
+    if (!device_is_sm100()) return FP8_ERR_DEVICE;
+    return launch_blockscaled_gemm_mx(A, sA, B, b_major, sB, sb_gran, M, N, K, D, out_dtype, ldd,
+                                      static_cast<cudaStream_t>(stream));
+}
+
 FP8FG_API int fp8_grouped_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB,
                                const int32_t* group_offsets, int G, int64_t M_total, int64_t N,
                                int64_t K, void* D, int out_dtype, void* stream)
@@ -249,7 +271,8 @@ FP8FG_API int fp8_get_status(void* stream)
 {
     const int a = read_and_clear_status(static_cast<cudaStream_t>(stream));
     const int b = read_and_clear_moe_status();
-    return a != FP8_OK ? a : b;
+    const int c = read_and_clear_mx_status();
+    return a != FP8_OK ? a : (b != FP8_OK ? b : c);
 }
 
 FP8FG_API const char* fp8_status_string(int code)
@@ -263,6 +286,7 @@ FP8FG_API const char* fp8_status_string(int code)
         case FP8_ERR_LAUNCH: return "FP8_ERR_LAUNCH: CUDA launch failed";
         case FP8_ERR_TIMEOUT: return "FP8_ERR_TIMEOUT: a device-side wait ran out of time";
         case FP8_ERR_DEVICE: return "FP8_ERR_DEVICE: no supported (sm_100) CUDA device";
+        case FP8_ERR_VALUE: return "FP8_ERR_VALUE: a scale is not a positive normal power of two";
         default: return "unknown fp8fg status";
     }
 }

@@ -16,10 +16,26 @@
 
 namespace fp8fg {
 
-// Record `code` in the library's status word (first error wins).  Defined,
-// together with the status word itself, in gemm.cu -- the only translation
-// unit whose kernels report device-side errors.
-__device__ void report_error(int code);
+// Status word of this kernel module.  Device code is compiled per source
+// file, so every source file that includes this header gets its own word
+// (internal linkage, module scope, never allocated); each such file exports
+// a reader, and fp8_get_status reads and clears them all.
+namespace {
+__device__ int g_module_status = 0;
+
+// Record `code` in this module's status word (first error wins).
+__device__ __forceinline__ void report_error(int code) { atomicCAS(&g_module_status, 0, code); }
+
+// Host: return and clear this module's status word (caller synchronised).
+inline int read_and_clear_module_status()
+{
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_module_status, sizeof(int)) != cudaSuccess) return FP8_ERR_DEVICE;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_module_status, &zero, sizeof(int)) != cudaSuccess) return FP8_ERR_DEVICE;
+    return v;
+}
+}  // namespace
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p)
 {
@@ -256,6 +272,29 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(uint32_t M, uint32_t N, ui
            | ((N >> 3) << 17)        // N / 8
            | ((M >> 4) << 24);       // M / 16
 }
+
+// ---------------------------------------------------------------- GEMM tiles
+
+// Persistent-GEMM tile order: bands of `band` m-blocks; inside a band n-blocks
+// outer, m-blocks inner, so the tiles resident at once share a few A
+// row-blocks and B column-blocks in L2.
+__device__ __forceinline__ void gemm_tile_coord(int64_t tile, int64_t nmb, int64_t nnb, int band,
+                                                int64_t& mb, int64_t& nb)
+{
+    const int64_t band_tiles = (int64_t)band * nnb;
+    const int64_t bi = tile / band_tiles;
+    const int64_t r = tile - bi * band_tiles;
+    const int64_t mb0 = bi * band;
+    const int64_t rows = (nmb - mb0 < band) ? (nmb - mb0) : band;
+    nb = r / rows;
+    mb = mb0 + r % rows;
+}
+
+// Host: 2-D uint8 tensor map [outer][inner], rows `row_bytes` apart, boxes of
+// box_inner x box_outer bytes, 128-byte swizzle, zero fill out of bounds
+// (defined in gemm.cu; false when the driver's encoder is unavailable).
+bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
 
 // ---------------------------------------------------------------- registers
 

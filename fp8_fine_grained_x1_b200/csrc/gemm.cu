@@ -37,11 +37,6 @@
 
 namespace fp8fg {
 
-// The library's status word (one per device; module-scope, not allocated).
-__device__ int g_status = 0;
-
-__device__ void report_error(int code) { atomicCAS(&g_status, 0, code); }
-
 namespace {
 
 constexpr int BM = 128;
@@ -77,21 +72,6 @@ struct GemmParams {
     int b_box_rows;                // rows of a K-major B box (128 or 256)
     uint64_t timeout_ns;
 };
-
-// Tile order: bands of BAND m-blocks; inside a band n-blocks outer, m-blocks
-// inner, so the tiles resident at once share a few A row-blocks and B
-// column-blocks in L2.
-__device__ __forceinline__ void tile_coord(int64_t tile, int64_t nmb, int64_t nnb, int64_t& mb,
-                                           int64_t& nb)
-{
-    const int64_t band_tiles = (int64_t)BAND * nnb;
-    const int64_t band = tile / band_tiles;
-    const int64_t r = tile - band * band_tiles;
-    const int64_t mb0 = band * BAND;
-    const int64_t rows = (nmb - mb0 < BAND) ? (nmb - mb0) : BAND;
-    nb = r / rows;
-    mb = mb0 + r % rows;
-}
 
 // Group of the 128-row block starting at row0: the largest e with
 // off[e] <= row0; -1 when row0 >= off[G] (rows outside every group).
@@ -141,7 +121,7 @@ __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, con
     bool ok = true;
     for (int64_t tile = blockIdx.x; ok && tile < nmb * nnb; tile += gridDim.x) {
         int64_t mb, nb;
-        tile_coord(tile, nmb, nnb, mb, nb);
+        gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
         const int64_t m0 = mb * BM, n0 = nb * BN;
         int g = 0;
         if (p.group_offsets) {
@@ -194,7 +174,7 @@ __device__ void run_mma(const GemmParams& p, uint8_t* smem, Shared& sh, int64_t 
     bool ok = true;
     for (int64_t tile = blockIdx.x; ok && tile < nmb * nnb; tile += gridDim.x) {
         int64_t mb, nb;
-        tile_coord(tile, nmb, nnb, mb, nb);
+        gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
         const int64_t n0 = nb * BN;
         if (p.group_offsets && find_group(sh.off, p.G, mb * BM) < 0) continue;
         const int64_t n_valid = (p.N - n0 < BN) ? (p.N - n0) : BN;
@@ -245,7 +225,7 @@ __device__ void run_promotion(const GemmParams& p, Shared& sh, int nmb, int nnb,
 
     for (int tile = blockIdx.x; tile < nmb * nnb; tile += gridDim.x) {
         int64_t mb64, nb64;
-        tile_coord(tile, nmb, nnb, mb64, nb64);
+        gemm_tile_coord(tile, nmb, nnb, BAND, mb64, nb64);
         const int mb = (int)mb64, nb = (int)nb64;
         const int m0 = mb * BM, n0 = nb * BN;
         int g = 0;
@@ -470,6 +450,25 @@ __global__ void k_selftest_wait(uint64_t timeout_ns)
 
 // ------------------------------------------------------------------ host side
 
+bool ensure_smem_attr()
+{
+    // once per device
+    static bool done[64] = {};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!done[dev]) {
+        if (cudaFuncSetAttribute(k_fp8_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)DYN_SMEM) != cudaSuccess)
+            return false;
+        done[dev] = true;
+    }
+    return true;
+}
+
+}  // namespace
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -505,25 +504,6 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-
-bool ensure_smem_attr()
-{
-    // once per device
-    static bool done[64] = {};
-    static std::mutex mu;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-    std::lock_guard<std::mutex> lk(mu);
-    if (!done[dev]) {
-        if (cudaFuncSetAttribute(k_fp8_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)DYN_SMEM) != cudaSuccess)
-            return false;
-        done[dev] = true;
-    }
-    return true;
-}
-
-}  // namespace
 
 int launch_blockscaled_gemm(const uint8_t* A, const float* sA, const uint8_t* B, int b_major,
                             const float* sB, int sb_gran, int64_t M, int64_t N, int64_t K,
@@ -573,15 +553,12 @@ cudaError_t launch_selftest_wait(cudaStream_t st)
     return cudaGetLastError();
 }
 
-// Synchronise, then read and clear the status word of the current device.
+// Synchronise, then read and clear this module's status word on the current
+// device.
 int read_and_clear_status(cudaStream_t st)
 {
     if (cudaStreamSynchronize(st) != cudaSuccess) return FP8_ERR_DEVICE;
-    int v = 0;
-    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return FP8_ERR_DEVICE;
-    const int zero = 0;
-    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return FP8_ERR_DEVICE;
-    return v;
+    return read_and_clear_module_status();
 }
 
 }  // namespace fp8fg

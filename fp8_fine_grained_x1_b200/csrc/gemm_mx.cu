@@ -1,0 +1,525 @@
+// gemm_mx.cu -- block-scaled E4M3 x E4M3 GEMM for power-of-two scales, with
+// the scaling done by the tensor cores (sm_100a:
+// tcgen05.mma.kind::mxf8f6f4.block_scale, UE8M0 scale factors in TMEM).
+//
+// What it computes is the same sum as gemm.cu -- D = sum over 128-element
+// K-blocks of scale_a * scale_b * (A_kb . B_kb) -- restricted to scales that
+// are integral powers of two ("5 Ways You can get More Deepseek While
+// Spending Less": power-of-2 scaling factors for some activations; the
+// gnrental.net post: the authors ask for Tensor Cores that take group scales
+// themselves and accumulate at higher precision, so partials need not leave
+// them).  A power of two is exactly a UE8M0 scale factor, so the multiply by
+// scale_a * scale_b happens inside the MMA: each tcgen05.mma of K = 32 reads
+// one scale per row of A and one per column of B from TMEM and accumulates
+// the scaled products into the FP32 accumulator.  No partial leaves the
+// tensor core until the tile's last K-block: there is no promotion step.
+//
+// Roles per CTA (persistent, one CTA per SM, 512 threads):
+//   warp 0      TMA producer: A / B tiles per K-block into a 4-stage ring
+//               (128-byte swizzle, no cluster multicast)
+//   warp 1      MMA issuer: 4 x block-scaled MMA (K = 32) per K-block into
+//               one TMEM accumulator, tcgen05.commit frees the stage
+//   warp 2      TMEM allocator
+//   warps 4-7   scale writers: per K-block, read the FP32 scales, take
+//               their biased exponents (UE8M0) and store them into the
+//               stage's scale-factor area of shared memory; the MMA thread
+//               copies them to TMEM (tcgen05.cp) in order with its MMAs
+//   warps 8-15  epilogue: tcgen05.ld the accumulator (two warps per lane
+//               quarter, 128 columns each), release it, convert and store
+// TMEM (512 columns): accumulator 0-255; per stage s a 16-column slot at
+// 256 + 16 s: SFA in its first 4 columns, SFB in columns 8-15.
+// Scale-factor layout (the tensor core's for M = 128, one scale per 32 K):
+// column c of the SFA slot holds, in lane 32 q + l, the scale of row
+// 32 c + l; column c of the SFB slot the scale of column 32 c + l; every
+// lane quarter q holds the same copy.  All four bytes of a column word are
+// the same scale, because one 128-element group covers all four K = 32
+// steps of a K-block, so whichever byte an MMA selects is the right one.
+// In shared memory each 128 rows (or columns) form one 512-byte block of 32
+// lines of 16 bytes: line l = the words of rows l, l + 32, l + 64, l + 96.
+// tcgen05.cp .32x128b.warpx4 moves line l to TMEM lane l of every quarter,
+// four columns wide -- exactly the layout above.  (Writing TMEM with
+// tcgen05.st from the scale warps instead measured 24 % tensor-pipe
+// activity: the stores and the MMAs contend for TMEM.)
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "fp8fg_device.cuh"
+#include "fp8fg_host.h"
+
+namespace fp8fg {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 128;
+constexpr int NS = 4;
+constexpr uint32_t A_BYTES = BM * BK;
+constexpr uint32_t B_BYTES = BN * BK;
+constexpr int NUM_THREADS = 512;
+constexpr int FIRST_SF_WARP = 4;
+constexpr int FIRST_EPI_WARP = 8;
+constexpr int NUM_SF_WARPS = 4;
+constexpr int NUM_EPI_WARPS = 8;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t SF_COL0 = BN;
+constexpr uint32_t SF_SLOT_COLS = 16;
+constexpr uint32_t SFB_OFF = 8;
+static_assert(SF_COL0 + NS * SF_SLOT_COLS <= TMEM_COLS, "scale slots exceed the allocation");
+constexpr int BAND = 16;
+constexpr int SF_AHEAD = 4;                 // K-blocks of scales each writer loads ahead
+constexpr uint32_t SFA_BYTES = 512;              // 128 rows x 4 bytes
+constexpr uint32_t SFB_BYTES = 1024;             // 256 columns x 4 bytes
+constexpr uint32_t SF_BYTES = SFA_BYTES + SFB_BYTES;
+constexpr uint32_t DYN_SMEM = 1024 + NS * (A_BYTES + B_BYTES + SF_BYTES);
+
+struct MxParams {
+    const float* sA;     // [K/128][M]
+    const float* sB;     // as for fp8_blockscaled_gemm
+    void* D;
+    int64_t M, N, K, ldd;
+    int b_major, sb_gran, out_dtype;
+    int b_box_rows;
+    uint64_t timeout_ns;
+};
+
+struct __align__(8) MxShared {
+    uint64_t full[NS];
+    uint64_t empty[NS];
+    uint64_t sf_full[NS];
+    uint64_t acc_full;
+    uint64_t acc_empty;
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// -------------------------------------------------------------- PTX helpers
+
+// Block-scaled MMA: D[tmem] (+)= (A * SFA) x (B * SFB), E4M3 operands from
+// shared memory, UE8M0 scale factors from TMEM, one CTA.
+__device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                         uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::
+            "r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// Instruction descriptor of the block-scaled kind: E4M3 x E4M3, UE8M0 scale
+// factors (bit 23), scale-factor ids 0, K = 32, A K-major; FP32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3(uint32_t M, uint32_t N, uint32_t b_mn_major)
+{
+    return (0u << 7)                 // A format: E4M3
+           | (0u << 10)              // B format: E4M3
+           | (b_mn_major << 16)      // B major
+           | ((N >> 3) << 17)        // N / 8
+           | (1u << 23)              // scale factors: UE8M0
+           | ((M >> 4) << 24);       // M / 16
+}
+
+// Copy 32 lines of 16 bytes (a 512-byte block at `saddr`, no swizzle) from
+// shared memory to TMEM: line l -> lane l of every lane quarter, four 32-bit
+// columns from `taddr`.  Issued by the MMA thread; executes in order with
+// the tcgen05.mma instructions it issues afterwards.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint32_t saddr)
+{
+    // descriptor: start >> 4; leading offset 16 B (unused: one 16-byte column);
+    // stride 128 B between groups of 8 lines; version 1; no swizzle
+    const uint64_t desc = (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)(16 >> 4) << 16) |
+                          ((uint64_t)(128 >> 4) << 32) | ((uint64_t)1 << 46);
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc)
+                 : "memory");
+}
+
+// Make this thread's shared-memory stores visible to the async proxy (TMA,
+// tcgen05.cp, tcgen05.mma operand reads).
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// UE8M0 code of a scale 2^e (-126 <= e <= 127): its biased exponent, copied
+// into all four bytes.  Anything that is not a positive normal power of two
+// sets `bad` and is replaced by 2^0.
+__device__ __forceinline__ uint32_t ue8m0_x4(float s, bool& bad)
+{
+    const uint32_t b = __float_as_uint(s);
+    const uint32_t e = b >> 23;                       // sign bit included: negative -> > 255
+    const bool ok = (b & 0x007FFFFFu) == 0u && e >= 1u && e <= 254u;
+    bad = bad || !ok;
+    return (ok ? e : 127u) * 0x01010101u;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi)
+{
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// One lane waits (bounded); the whole warp learns the outcome, so the warp's
+// .sync.aligned tcgen05 instructions are never reached by part of it.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t timeout_ns, int lane)
+{
+    int ok = 1;
+    if (lane == 0) ok = mbar_wait(bar, parity, abort, timeout_ns) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// ------------------------------------------------------------------ roles
+
+__device__ void mx_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const MxParams& p,
+                            uint8_t* smem, MxShared& sh, int64_t nmb, int64_t nnb, int64_t nkb)
+{
+    volatile int* abort = &sh.abort;
+    int64_t it = 0;
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; ok && tile < nmb * nnb; tile += gridDim.x) {
+        int64_t mb, nb;
+        gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
+        const int64_t m0 = mb * BM, n0 = nb * BN;
+        const int64_t n_valid = (p.N - n0 < BN) ? (p.N - n0) : BN;
+        const uint32_t b_bytes = (p.b_major == FP8_B_KMAJOR) ? (uint32_t)p.b_box_rows * BK
+                                                             : (uint32_t)n_valid * BK;
+        for (int64_t kb = 0; kb < nkb; ++kb) {
+            const int s = (int)(it % NS);
+            const uint32_t ph = (uint32_t)((it / NS) & 1);
+            if (!mbar_wait(&sh.empty[s], ph ^ 1u, abort, p.timeout_ns)) {
+                ok = false;
+                break;
+            }
+            ++it;
+            mbar_arrive_expect_tx(&sh.full[s], A_BYTES + b_bytes);
+            uint8_t* a_dst = smem + s * A_BYTES;
+            uint8_t* b_dst = smem + NS * A_BYTES + s * B_BYTES;
+            tma_load_2d(a_dst, tmA, &sh.full[s], (int32_t)(kb * BK), (int32_t)m0);
+            if (p.b_major == FP8_B_KMAJOR) {
+                tma_load_2d(b_dst, tmB, &sh.full[s], (int32_t)(kb * BK), (int32_t)n0);
+            } else {
+                tma_load_2d(b_dst, tmB, &sh.full[s], (int32_t)n0, (int32_t)(kb * BK));
+                if (n_valid > 128)
+                    tma_load_2d(b_dst + 128 * BK, tmB, &sh.full[s], (int32_t)(n0 + 128),
+                                (int32_t)(kb * BK));
+            }
+        }
+    }
+    // every copy issued lands before the CTA exits
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+        const int64_t count = it > s ? (it - s + NS - 1) / NS : 0;
+        if (count) mbar_wait_drain(&sh.full[s], (uint32_t)((count - 1) & 1), p.timeout_ns);
+    }
+}
+
+__device__ void mx_mma(const MxParams& p, uint8_t* smem, MxShared& sh, int64_t nmb, int64_t nnb,
+                       int64_t nkb)
+{
+    volatile int* abort = &sh.abort;
+    const uint32_t a_base = smem_u32(smem);
+    const uint32_t b_base = a_base + NS * A_BYTES;
+    const uint32_t sf_base = b_base + NS * B_BYTES;
+    const uint32_t tmem = sh.tmem_base;
+    int64_t it = 0;
+    uint32_t tcount = 0;
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; ok && tile < nmb * nnb; tile += gridDim.x, ++tcount) {
+        int64_t mb, nb;
+        gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
+        const int64_t n0 = nb * BN;
+        const int64_t n_valid = (p.N - n0 < BN) ? (p.N - n0) : BN;
+        const uint32_t idesc = idesc_mx_e4m3(BM, (uint32_t)n_valid, (uint32_t)p.b_major);
+        // the epilogue has read the previous tile's accumulator
+        if (!mbar_wait(&sh.acc_empty, (tcount & 1u) ^ 1u, abort, p.timeout_ns)) break;
+        tc_fence_after();
+        for (int64_t kb = 0; kb < nkb; ++kb, ++it) {
+            const int s = (int)(it % NS);
+            const uint32_t ph = (uint32_t)((it / NS) & 1);
+            if (!mbar_wait(&sh.sf_full[s], ph, abort, p.timeout_ns) ||
+                !mbar_wait(&sh.full[s], ph, abort, p.timeout_ns)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t a_addr = a_base + s * A_BYTES;
+            const uint32_t b_addr = b_base + s * B_BYTES;
+            const uint32_t sf_addr = sf_base + s * SF_BYTES;
+            const uint32_t sfa = tmem + SF_COL0 + (uint32_t)s * SF_SLOT_COLS;
+            tmem_cp_32x128b_x4(sfa, sf_addr);                               // SFA, rows 0-127
+            tmem_cp_32x128b_x4(sfa + SFB_OFF, sf_addr + SFA_BYTES);         // SFB, columns 0-127
+            tmem_cp_32x128b_x4(sfa + SFB_OFF + 4, sf_addr + SFA_BYTES + 512);   // columns 128-255
+#pragma unroll
+            for (int k = 0; k < BK / 32; ++k) {
+                const uint64_t adesc = smem_desc_sw128(a_addr + k * 32, 16, 1024);
+                const uint64_t bdesc = (p.b_major == FP8_B_KMAJOR)
+                                           ? smem_desc_sw128(b_addr + k * 32, 16, 1024)
+                                           : smem_desc_sw128(b_addr + k * 32 * 128, 128 * BK, 1024);
+                mma_mxf8(tmem, adesc, bdesc, idesc, sfa, sfa + SFB_OFF, (kb | k) ? 1u : 0u);
+            }
+            mma_commit(&sh.empty[s]);        // stage and scale slot free once these are done
+        }
+        if (!ok) break;
+        mma_commit(&sh.acc_full);            // the tile's sum is complete
+    }
+    mma_commit(&sh.drain);
+    mbar_wait_drain(&sh.drain, 0, p.timeout_ns);
+}
+
+// Scales of K-block kb handled by scale-writer thread t (0..127): row t of
+// the tile's A block and columns t, t + 128 of its B block; 1 outside the
+// matrix.
+struct SfRegs {
+    float a;
+    float b[2];
+};
+
+__device__ __forceinline__ void load_sf(const MxParams& p, int64_t m0, int64_t n0, int64_t kb,
+                                        int64_t nkb, int t, SfRegs& r)
+{
+    const int64_t m = m0 + t;
+    r.a = m < p.M ? __ldg(p.sA + kb * p.M + m) : 1.0f;
+    const int64_t nnb128 = p.N / 128;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const int64_t n = n0 + t + 128 * j;
+        float v = 1.0f;
+        if (n < p.N) {
+            if (p.sb_gran == 1)
+                v = __ldg(p.sB + kb * p.N + n);
+            else if (p.b_major == FP8_B_KMAJOR)
+                v = __ldg(p.sB + (n / 128) * nkb + kb);
+            else
+                v = __ldg(p.sB + kb * nnb128 + n / 128);
+        }
+        r.b[j] = v;
+    }
+}
+
+// Byte offset of row (or column) i of a 128-row block in its 512-byte block:
+// line i % 32, word i / 32.
+__device__ __forceinline__ uint32_t sf_offset(int i) { return 16u * (uint32_t)(i & 31) + 4u * (uint32_t)(i >> 5); }
+
+__device__ void mx_scale_writer(const MxParams& p, uint8_t* smem, MxShared& sh, int64_t nmb,
+                                int64_t nnb, int64_t nkb, int warp, int lane)
+{
+    volatile int* abort = &sh.abort;
+    const int t = (warp - FIRST_SF_WARP) * 32 + lane;          // 0..127
+    uint8_t* sf_base = smem + NS * (A_BYTES + B_BYTES);
+    const uint32_t off_a = sf_offset(t);
+    const uint32_t off_b0 = SFA_BYTES + sf_offset(t);
+    const uint32_t off_b1 = SFA_BYTES + 512 + sf_offset(t);
+    int64_t it = 0;
+    bool ok = true, bad = false;
+    for (int64_t tile = blockIdx.x; ok && tile < nmb * nnb; tile += gridDim.x) {
+        int64_t mb, nb;
+        gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
+        const int64_t m0 = mb * BM, n0 = nb * BN;
+        // SF_AHEAD K-blocks of scale loads in flight per thread
+        SfRegs ring[SF_AHEAD];
+#pragma unroll
+        for (int u = 0; u < SF_AHEAD; ++u)
+            if (u < nkb) load_sf(p, m0, n0, u, nkb, t, ring[u]);
+        for (int64_t kb0 = 0; ok && kb0 < nkb; kb0 += SF_AHEAD) {
+#pragma unroll
+            for (int u = 0; u < SF_AHEAD; ++u) {
+                const int64_t kb = kb0 + u;
+                if (ok && kb < nkb) {            // warp-uniform
+                    const uint32_t wa = ue8m0_x4(ring[u].a, bad);
+                    const uint32_t wb0 = ue8m0_x4(ring[u].b[0], bad);
+                    const uint32_t wb1 = ue8m0_x4(ring[u].b[1], bad);
+                    if (kb + SF_AHEAD < nkb) load_sf(p, m0, n0, kb + SF_AHEAD, nkb, t, ring[u]);
+                    const int s = (int)(it % NS);
+                    const uint32_t ph = (uint32_t)((it / NS) & 1);
+                    // the copies and MMAs that last read this stage have completed
+                    if (warp_wait(&sh.empty[s], ph ^ 1u, abort, p.timeout_ns, lane)) {
+                        ++it;
+                        uint8_t* sf = sf_base + s * SF_BYTES;
+                        *reinterpret_cast<uint32_t*>(sf + off_a) = wa;
+                        *reinterpret_cast<uint32_t*>(sf + off_b0) = wb0;
+                        *reinterpret_cast<uint32_t*>(sf + off_b1) = wb1;
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sh.sf_full[s]);
+                    } else {
+                        ok = false;
+                    }
+                }
+            }
+        }
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) report_error(FP8_ERR_VALUE);
+}
+
+__device__ void mx_epilogue(const MxParams& p, MxShared& sh, int64_t nmb, int64_t nnb, int warp,
+                            int lane)
+{
+    volatile int* abort = &sh.abort;
+    const int ew = warp - FIRST_EPI_WARP;       // 0..7
+    const int q = warp & 3;
+    const int col0 = (ew >> 2) * 128;
+    const int row = q * 32 + lane;
+    const uint32_t taddr0 = sh.tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)col0;
+    uint32_t tcount = 0;
+    for (int64_t tile = blockIdx.x; tile < nmb * nnb; tile += gridDim.x, ++tcount) {
+        int64_t mb, nb;
+        gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
+        const int64_t m = mb * BM + row;
+        const int64_t n0 = nb * BN + col0;
+        const bool active = n0 < p.N;           // warp-uniform
+        const bool row_ok = m < p.M;
+        if (!warp_wait(&sh.acc_full, tcount & 1u, abort, p.timeout_ns, lane)) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            if (active) {
+                tmem_ld32(taddr0 + (uint32_t)(c * 32), r);
+                tmem_ld_wait();
+            }
+            if (c == 3) {                        // accumulator no longer needed
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sh.acc_empty);
+            }
+            if (!(active && row_ok)) continue;
+            if (p.out_dtype == FP8_OUT_BF16) {
+                uint4* d = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.D) + m * p.ldd +
+                                                    n0 + c * 32);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    uint4 w;
+                    w.x = pack_bf16x2_rn(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+                    w.y = pack_bf16x2_rn(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+                    w.z = pack_bf16x2_rn(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+                    w.w = pack_bf16x2_rn(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+                    d[v] = w;
+                }
+            } else {
+                uint4* d = reinterpret_cast<uint4*>(static_cast<float*>(p.D) + m * p.ldd + n0 + c * 32);
+#pragma unroll
+                for (int v = 0; v < 8; ++v)
+                    d[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    k_fp8_gemm_mx(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                  const MxParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ MxShared sh;
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t nmb = (p.M + BM - 1) / BM;
+    const int64_t nnb = (p.N + BN - 1) / BN;
+    const int64_t nkb = p.K / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&sh.full[s], 1);
+            mbar_init(&sh.empty[s], 1);
+            mbar_init(&sh.sf_full[s], NUM_SF_WARPS);
+        }
+        mbar_init(&sh.acc_full, 1);
+        mbar_init(&sh.acc_empty, NUM_EPI_WARPS);
+        mbar_init(&sh.drain, 1);
+        sh.abort = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 2) {
+        tmem_alloc(&sh.tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    if (warp == 0) {
+        if (lane == 0) mx_producer(&tmA, &tmB, p, smem, sh, nmb, nnb, nkb);
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) mx_mma(p, smem, sh, nmb, nnb, nkb);
+        __syncwarp();
+    } else if (warp >= FIRST_SF_WARP && warp < FIRST_SF_WARP + NUM_SF_WARPS) {
+        mx_scale_writer(p, smem, sh, nmb, nnb, nkb, warp, lane);
+    } else if (warp >= FIRST_EPI_WARP) {
+        mx_epilogue(p, sh, nmb, nnb, warp, lane);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 2) tmem_dealloc(sh.tmem_base, TMEM_COLS);
+}
+
+bool ensure_mx_smem_attr()
+{
+    static bool done[64] = {};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!done[dev]) {
+        if (cudaFuncSetAttribute(k_fp8_gemm_mx, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)DYN_SMEM) != cudaSuccess)
+            return false;
+        done[dev] = true;
+    }
+    return true;
+}
+
+}  // namespace
+
+int launch_blockscaled_gemm_mx(const uint8_t* A, const float* sA, const uint8_t* B, int b_major,
+                               const float* sB, int sb_gran, int64_t M, int64_t N, int64_t K,
+                               void* D, int out_dtype, int64_t ldd, cudaStream_t st)
+{
+    if (M == 0) return FP8_OK;
+    CUtensorMap tmA, tmB;
+    const int b_box_rows = N >= BN ? BN : (int)N;
+    if (!make_map(&tmA, A, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, BM)) return FP8_ERR_LAUNCH;
+    const bool okB = (b_major == FP8_B_KMAJOR)
+                         ? make_map(&tmB, B, (uint64_t)K, (uint64_t)N, (uint64_t)K, BK,
+                                    (uint32_t)b_box_rows)
+                         : make_map(&tmB, B, (uint64_t)N, (uint64_t)K, (uint64_t)N, 128, BK);
+    if (!okB || !ensure_mx_smem_attr()) return FP8_ERR_LAUNCH;
+
+    MxParams p;
+    p.sA = sA;
+    p.sB = sB;
+    p.D = D;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.ldd = ldd;
+    p.b_major = b_major;
+    p.sb_gran = sb_gran;
+    p.out_dtype = out_dtype;
+    p.b_box_rows = b_box_rows;
+    p.timeout_ns = wait_timeout_ns();
+
+    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int sms = device_sm_count();
+    const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
+    k_fp8_gemm_mx<<<grid, NUM_THREADS, DYN_SMEM, st>>>(tmA, tmB, p);
+    return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_LAUNCH;
+}
+
+int read_and_clear_mx_status() { return read_and_clear_module_status(); }
+
+}  // namespace fp8fg

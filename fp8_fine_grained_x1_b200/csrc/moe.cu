@@ -35,8 +35,6 @@ namespace {
 
 constexpr int kPairsPerChunk = 1024;
 
-// Records a malformed routing entry / capacity overflow (first error wins).
-__device__ int g_moe_status = 0;
 
 // Fixed dispatch scratch for the non-allocating entry point (one per device
 // context).  Every entry a dispatch reads is written earlier in the same
@@ -85,7 +83,7 @@ __global__ void __launch_bounds__(1024) k_moe_scan(int32_t* __restrict__ ws, int
             acc += padded[j];
         }
         base[G] = (int32_t)(acc < 0x7FFFFFFF ? acc : 0x7FFFFFFF);
-        if (acc > M_cap) atomicCAS(&g_moe_status, 0, FP8_ERR_SHAPE);
+        if (acc > M_cap) report_error(FP8_ERR_SHAPE);
     }
     __syncthreads();
     for (int j = threadIdx.x; j <= G; j += blockDim.x) offsets[j] = base[j];
@@ -109,7 +107,7 @@ __global__ void __launch_bounds__(32) k_moe_rank(const int32_t* __restrict__ top
         const bool live = idx < P;
         int32_t e = live ? topk[idx] : -1;
         const bool ok = live && e >= 0 && e < G;
-        if (live && !ok) atomicCAS(&g_moe_status, 0, FP8_ERR_SHAPE);
+        if (live && !ok) report_error(FP8_ERR_SHAPE);
         if (!ok) e = -1 - lane;                 // unique key: never matches another lane
         const unsigned same = __match_any_sync(0xffffffffu, e);
         const unsigned below = same & ((1u << lane) - 1u);
@@ -120,7 +118,7 @@ __global__ void __launch_bounds__(32) k_moe_rank(const int32_t* __restrict__ top
         __syncwarp();
         if (live) {
             const bool fits = ok && pos >= 0 && pos < M_cap;
-            if (ok && !fits) atomicCAS(&g_moe_status, 0, FP8_ERR_SHAPE);
+            if (ok && !fits) report_error(FP8_ERR_SHAPE);
             token_row[idx] = fits ? pos : -1;
             if (fits) row_token[pos] = (int32_t)(idx / k);
         }
@@ -267,13 +265,8 @@ cudaError_t moe_static_workspace(int32_t** ws)
     return cudaSuccess;
 }
 
-int read_and_clear_moe_status()
-{
-    int v = 0;
-    if (cudaMemcpyFromSymbol(&v, g_moe_status, sizeof(int)) != cudaSuccess) return FP8_ERR_DEVICE;
-    const int zero = 0;
-    if (cudaMemcpyToSymbol(g_moe_status, &zero, sizeof(int)) != cudaSuccess) return FP8_ERR_DEVICE;
-    return v;
-}
+// Malformed routing entries and capacity overflows are recorded in this
+// module's status word.
+int read_and_clear_moe_status() { return read_and_clear_module_status(); }
 
 }  // namespace fp8fg

@@ -21,12 +21,18 @@ Dgrad and Wgrad all run in FP8; why-be.co.kr / cameseeing.com posts and
 grouping; gnrental.net post: BF16 or FP32 GEMM outputs.)
 
 `kernel_calls` on each step counts the kernels one call launches.
+
+With scale_mode=SCALE_POW2 the dense steps accept tensor_core_scaling=True:
+the GEMM then applies the power-of-two scales inside the tensor cores
+(fp8_blockscaled_gemm_pow2, UE8M0 block scaling) instead of promoting every
+128-K partial in software.
 """
 from __future__ import annotations
 
 import torch
 
-from . import (B_KMAJOR, B_MNMAJOR, SCALE_FP32, fp8_blockscaled_gemm, fp8_grouped_gemm,
+from . import (B_KMAJOR, B_MNMAJOR, SCALE_FP32, SCALE_POW2, fp8_blockscaled_gemm,
+               fp8_blockscaled_gemm_pow2, fp8_grouped_gemm,
                fp8_moe_combine, fp8_moe_dispatch, fp8_moe_dispatch_workspace_bytes,
                fp8_quant_act_128x1, fp8_quant_act_1x128, fp8_quant_w_128x128,
                fp8_requant_1x128_to_128x1, moe_capacity)
@@ -36,14 +42,24 @@ def _empty(shape, dtype, device):
     return torch.empty(shape, dtype=dtype, device=device)
 
 
+def _gemm_fn(scale_mode, tensor_core_scaling):
+    if not tensor_core_scaling:
+        return fp8_blockscaled_gemm
+    if scale_mode != SCALE_POW2:
+        raise ValueError("tensor-core scaling needs power-of-two scales (SCALE_POW2)")
+    return fp8_blockscaled_gemm_pow2
+
+
 class FpropStep:
     kernel_calls = 3
 
-    def __init__(self, x, w, out_dtype=torch.bfloat16, scale_mode=SCALE_FP32):
+    def __init__(self, x, w, out_dtype=torch.bfloat16, scale_mode=SCALE_FP32,
+                 tensor_core_scaling=False):
         M, K = x.shape
         N = w.shape[0]
         d = x.device
         self.x, self.w, self.mode = x, w, scale_mode
+        self._gemm = _gemm_fn(scale_mode, tensor_core_scaling)
         self.qx, self.sx = _empty((M, K), torch.uint8, d), _empty((K // 128, M), torch.float32, d)
         self.qw, self.sw = _empty((N, K), torch.uint8, d), _empty((N // 128, K // 128), torch.float32, d)
         self.y = _empty((M, N), out_dtype, d)
@@ -55,7 +71,7 @@ class FpropStep:
         fp8_quant_w_128x128(self.w, self.qw, self.sw, self.mode, stream)
 
     def gemm(self, stream=None):
-        fp8_blockscaled_gemm(self.qx, self.sx, self.qw, self.sw, self.y, B_KMAJOR, 128, stream)
+        self._gemm(self.qx, self.sx, self.qw, self.sw, self.y, B_KMAJOR, 128, stream)
 
     def __call__(self, stream=None):
         self.quantize(stream)
@@ -66,12 +82,14 @@ class FpropStep:
 class DgradStep:
     kernel_calls = 3
 
-    def __init__(self, dy, w, out_dtype=torch.bfloat16, scale_mode=SCALE_FP32):
+    def __init__(self, dy, w, out_dtype=torch.bfloat16, scale_mode=SCALE_FP32,
+                 tensor_core_scaling=False):
         M, N_out = dy.shape
         N_out2, K_in = w.shape
         assert N_out == N_out2
         d = dy.device
         self.dy, self.w, self.mode = dy, w, scale_mode
+        self._gemm = _gemm_fn(scale_mode, tensor_core_scaling)
         self.qdy = _empty((M, N_out), torch.uint8, d)
         self.sdy = _empty((N_out // 128, M), torch.float32, d)
         self.qw = _empty((N_out, K_in), torch.uint8, d)
@@ -87,7 +105,7 @@ class DgradStep:
     def gemm(self, stream=None):
         # B = W stored [K = N_out][N = K_in]: MN-major; its block scales
         # sW[N_out/128][K_in/128] are [K/128][N/128] in GEMM terms.
-        fp8_blockscaled_gemm(self.qdy, self.sdy, self.qw, self.sw, self.dx, B_MNMAJOR, 128, stream)
+        self._gemm(self.qdy, self.sdy, self.qw, self.sw, self.dx, B_MNMAJOR, 128, stream)
 
     def __call__(self, stream=None):
         self.quantize(stream)
@@ -98,12 +116,13 @@ class DgradStep:
 class WgradStep:
     kernel_calls = 3
 
-    def __init__(self, x, dy, scale_mode=SCALE_FP32):
+    def __init__(self, x, dy, scale_mode=SCALE_FP32, tensor_core_scaling=False):
         T, C_in = x.shape
         T2, C_out = dy.shape
         assert T == T2
         d = x.device
         self.x, self.dy, self.mode = x, dy, scale_mode
+        self._gemm = _gemm_fn(scale_mode, tensor_core_scaling)
         self.qxT = _empty((C_in, T), torch.uint8, d)
         self.sx = _empty((T // 128, C_in), torch.float32, d)
         self.qdyT = _empty((C_out, T), torch.uint8, d)
@@ -117,7 +136,7 @@ class WgradStep:
         fp8_quant_act_128x1(self.x, self.qxT, self.sx, self.mode, stream)
 
     def gemm(self, stream=None):
-        fp8_blockscaled_gemm(self.qdyT, self.sdy, self.qxT, self.sx, self.dw, B_KMAJOR, 1, stream)
+        self._gemm(self.qdyT, self.sdy, self.qxT, self.sx, self.dw, B_KMAJOR, 1, stream)
 
     def __call__(self, stream=None):
         self.quantize(stream)

@@ -64,7 +64,9 @@ enum fp8_status {
     FP8_ERR_DTYPE = 4,    /* unknown dtype / mode / major / granularity enum     */
     FP8_ERR_LAUNCH = 5,   /* the CUDA launch failed (cudaGetLastError)           */
     FP8_ERR_TIMEOUT = 6,  /* a bounded device-side wait gave up (status word)    */
-    FP8_ERR_DEVICE = 7    /* no CUDA device, or not an sm_100 (B200-class) GPU   */
+    FP8_ERR_DEVICE = 7,   /* no CUDA device, or not an sm_100 (B200-class) GPU   */
+    FP8_ERR_VALUE = 8     /* a scale given to fp8_blockscaled_gemm_pow2 is not a
+                             positive normal power of two (status word)          */
 };
 
 enum { FP8_IN_BF16 = 0, FP8_IN_FP32 = 1 };          /* quantizer input dtype   */
@@ -168,6 +170,24 @@ int fp8_quant_w_128x128(const void* w, int in_dtype, int64_t N, int64_t K, int64
 int fp8_blockscaled_gemm(const uint8_t* A, const float* sA, const uint8_t* B, int b_major,
                          const float* sB, int sb_gran, int64_t M, int64_t N, int64_t K, void* D,
                          int out_dtype, int64_t ldd, void* stream);
+
+/*
+ * fp8_blockscaled_gemm for power-of-two scales (FP8_SCALE_POW2 quantizers;
+ * [P1]: integral power-of-2 scaling factors), with the scaling done inside
+ * the tensor cores: each scale 2^e becomes the UE8M0 block-scale factor of
+ * a tcgen05.mma.kind::mxf8f6f4.block_scale, so the per-128-K partials are
+ * accumulated in the MMA's FP32 accumulator with their scales applied
+ * ([P5]: the hardware ask for Tensor Cores that take group scales and keep
+ * full-precision accumulation), and no partial is promoted by software.
+ * The result is the same sum as fp8_blockscaled_gemm's (up to rounding
+ * order).  Arguments, layouts, sizes and errors as fp8_blockscaled_gemm;
+ * additionally every sA / sB value must be 2^e with -126 <= e <= 127: any
+ * other value is used as 1 and reported as FP8_ERR_VALUE through the status
+ * word.
+ */
+int fp8_blockscaled_gemm_pow2(const uint8_t* A, const float* sA, const uint8_t* B, int b_major,
+                              const float* sB, int sb_gran, int64_t M, int64_t N, int64_t K,
+                              void* D, int out_dtype, int64_t ldd, void* stream);
 
 /*
  * Grouped (MoE expert) block-scaled GEMM: rows [off[e], off[e+1]) of A are

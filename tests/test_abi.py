@@ -50,7 +50,7 @@ def test_library_exports_exactly_the_header(lib):
 
 
 def test_status_strings(lib):
-    for code in range(8):
+    for code in range(9):
         assert fg.status_string(code).startswith("FP8_")
     assert "unknown" in fg.status_string(99)
 
@@ -101,9 +101,9 @@ def test_quant_128x1_and_w_validation(lib):
 
 
 def g(lib, *, A=FAKE, sA=FAKE2, B=FAKE3, bm=0, sB=FAKE4, gran=128, M=256, N=256, K=512,
-      D=FAKE5, od=0, ldd=None):
-    return lib.fp8_blockscaled_gemm(A, sA, B, bm, sB, gran, M, N, K, D, od,
-                                    N if ldd is None else ldd, None)
+      D=FAKE5, od=0, ldd=None, fn=None):
+    fn = lib.fp8_blockscaled_gemm if fn is None else fn
+    return fn(A, sA, B, bm, sB, gran, M, N, K, D, od, N if ldd is None else ldd, None)
 
 
 def test_gemm_validation(lib):
@@ -123,6 +123,35 @@ def test_gemm_validation(lib):
     assert g(lib, gran=128, sB=FAKE4 + 4) not in (fg.FP8_ERR_ALIGN,)
     assert g(lib, od=fg.OUT_BF16, ldd=260) == fg.FP8_ERR_ALIGN   # 520-B rows
     assert g(lib) in (fg.FP8_ERR_DEVICE, fg.FP8_OK)
+
+
+def test_gemm_pow2_validation(lib):
+    def gp(**kw):
+        return g(lib, fn=lib.fp8_blockscaled_gemm_pow2, **kw)
+    assert gp(od=5) == fg.FP8_ERR_DTYPE
+    assert gp(gran=1, bm=fg.B_MNMAJOR) == fg.FP8_ERR_DTYPE
+    assert gp(N=200) == fg.FP8_ERR_SHAPE
+    assert gp(K=130) == fg.FP8_ERR_SHAPE
+    assert gp(M=0, A=0, sA=0, B=0, sB=0, D=0) == fg.FP8_OK
+    assert gp(D=0) == fg.FP8_ERR_NULL
+    assert gp(A=FAKE + 16 + 8) == fg.FP8_ERR_ALIGN
+    assert gp(gran=1, sB=FAKE4 + 4) in (fg.FP8_ERR_DEVICE, fg.FP8_OK)   # scalar scale loads
+    assert gp() in (fg.FP8_ERR_DEVICE, fg.FP8_OK)
+
+
+def test_requant_validation(lib):
+    def rq(q=FAKE, ldq=256, sA=FAKE3, T=256, C=256, qT=FAKE2, ldqT=256, s=FAKE4, mode=fg.SCALE_FP32):
+        return lib.fp8_requant_1x128_to_128x1(q, ldq, sA, T, C, qT, ldqT, s, mode, None)
+    assert rq(mode=7) == fg.FP8_ERR_DTYPE
+    assert rq(T=200) == fg.FP8_ERR_SHAPE
+    assert rq(C=200, ldq=256) == fg.FP8_ERR_SHAPE                # channels in 128-blocks
+    assert rq(ldq=128) == fg.FP8_ERR_SHAPE
+    assert rq(ldqT=128) == fg.FP8_ERR_SHAPE
+    assert rq(C=0) == fg.FP8_OK
+    assert rq(sA=0) == fg.FP8_ERR_NULL
+    assert rq(ldq=264) == fg.FP8_ERR_ALIGN
+    assert rq(q=FAKE + 8) == fg.FP8_ERR_ALIGN
+    assert rq() in (fg.FP8_ERR_DEVICE, fg.FP8_OK)
 
 
 def test_grouped_validation(lib):

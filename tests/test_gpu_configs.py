@@ -101,6 +101,38 @@ def test_wgrad_token_axis_groups(mode):
     assert_gemm_close(d2h(dw)[pts[:, 0], pts[:, 1]], ref, tol, False, f"wgrad mode={mode}")
 
 
+def test_wgrad_pow2_scaled_in_tensor_cores():
+    wl = synth.wgrad()
+    step = linear.WgradStep(wl["x"].to(dev()), wl["dy"].to(dev()), scale_mode=fg.SCALE_POW2,
+                            tensor_core_scaling=True)
+    dw = step()
+    torch.cuda.synchronize()
+    assert fg.fp8_get_status() == fg.FP8_OK
+    qxT, sx = oracle.quant_act_128x1(_bits(wl["x"]), fg.SCALE_POW2)
+    qdyT, sdy = oracle.quant_act_128x1(_bits(wl["dy"]), fg.SCALE_POW2)
+    assert np.array_equal(step.qxT.cpu().numpy(), qxT) and np.array_equal(step.sx.cpu().numpy(), sx)
+    M, N = dw.shape
+    pts = _points(M, N, 6, rows=_edges(M, 128), cols=_edges(N, 256))
+    ref, tol = oracle.gemm_points(qdyT, sdy, qxT, sx, pts, sb_gran=1)
+    assert_gemm_close(d2h(dw)[pts[:, 0], pts[:, 1]], ref, tol, False, "wgrad pow2 tensor-core")
+
+
+def test_fprop_pow2_scaled_in_tensor_cores():
+    wl = synth.fprop()
+    step = linear.FpropStep(wl["x"].to(dev()), wl["w"].to(dev()), scale_mode=fg.SCALE_POW2,
+                            tensor_core_scaling=True)
+    y = step()
+    torch.cuda.synchronize()
+    assert fg.fp8_get_status() == fg.FP8_OK
+    qx, sx = oracle.quant_act_1x128(_bits(wl["x"]), fg.SCALE_POW2)
+    qw, sw = oracle.quant_w_128x128(_bits(wl["w"]), fg.SCALE_POW2)
+    assert np.array_equal(step.qx.cpu().numpy(), qx) and np.array_equal(step.qw.cpu().numpy(), qw)
+    M, N = y.shape
+    pts = _points(M, N, 7, rows=_edges(M, 128), cols=_edges(N, 256))
+    ref, tol = oracle.gemm_points(qx, sx, qw, sw, pts)
+    assert_gemm_close(d2h(y)[pts[:, 0], pts[:, 1]], ref, tol, True, "fprop pow2 tensor-core")
+
+
 def test_wgrad_from_cached_fp8_activations():
     """Wgrad with X taken from its cached 1x128 FP8 form (the forward's cache
     is made by the oracle here), requantized to 128x1 on the GPU."""

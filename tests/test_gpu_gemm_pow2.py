@@ -1,0 +1,89 @@
+"""GPU parity of fp8_blockscaled_gemm_pow2 (power-of-two scales applied by the
+tensor cores' UE8M0 block scaling) against the CPU oracle's FP64 block-scaled
+sum, within the same bound as the software-promoted GEMM: FP32 out
+|gpu - ref| <= 1e-4 * sum_k |s_a s_b a_k b_k|, BF16 out plus half a BF16 ulp.
+Operands are quantized by the oracle in power-of-two mode.
+"""
+import numpy as np
+import pytest
+import torch
+
+import fp8_fine_grained_x1_b200 as fg
+import oracle
+from fp8_fine_grained_x1_b200 import synth
+
+from gpu_util import assert_gemm_close, d2h, dev, to_dev
+
+pytestmark = pytest.mark.gpu
+P2 = oracle.SCALE_POW2
+
+
+def _operands(M, N, K, seed, b_major=oracle.B_KMAJOR):
+    x = synth.activations(M, K, seed=seed, outlier_seed=seed + 1).float().numpy()
+    w = synth.normal((N, K), 0.02, seed + 2).float().numpy()
+    qa, sa = oracle.quant_act_1x128(x, P2)
+    qw, sw = oracle.quant_w_128x128(w, P2)
+    if b_major == oracle.B_MNMAJOR:
+        # a weight stored [K][N] (the Dgrad orientation): quantize W^T in
+        # 128x128 blocks; its scales are then [K/128][N/128]
+        qw, sw = oracle.quant_w_128x128(np.ascontiguousarray(w.T), P2)
+    return qa, sa, qw, sw
+
+
+def _run(qa, sa, qb, sb, N, b_major=fg.B_KMAJOR, gran=128, out=torch.float32):
+    M = qa.shape[0]
+    D = torch.full((M, N), float("nan"), dtype=out, device=dev())
+    fg.fp8_blockscaled_gemm_pow2(to_dev(qa), to_dev(sa), to_dev(qb), to_dev(sb), D, b_major, gran)
+    torch.cuda.synchronize()
+    assert fg.fp8_get_status() == fg.FP8_OK
+    return d2h(D)
+
+
+@pytest.mark.parametrize("out", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 512), (200, 384, 640), (384, 512, 1024)])
+def test_pow2_gemm_kmajor_full_output(M, N, K, out):
+    qa, sa, qw, sw = _operands(M, N, K, seed=M + N)
+    got = _run(qa, sa, qw, sw, N, out=out)
+    ref, tol = oracle.gemm_full(qa, sa, qw, sw)
+    assert_gemm_close(got, ref, tol, out == torch.bfloat16, f"pow2 {M}x{N}x{K}")
+
+
+def test_pow2_gemm_mnmajor_weight():
+    M, N, K = 256, 384, 512
+    qa, sa, qw, sw = _operands(M, N, K, seed=5, b_major=oracle.B_MNMAJOR)
+    got = _run(qa, sa, qw, sw, N, b_major=fg.B_MNMAJOR, out=torch.bfloat16)
+    ref, tol = oracle.gemm_full(qa, sa, qw, sw, b_major=oracle.B_MNMAJOR)
+    assert_gemm_close(got, ref, tol, True, "pow2 MN-major")
+
+
+def test_pow2_gemm_per_column_scales():
+    """Wgrad form: both operands 128x1 along the inner (token) axis."""
+    T, C_out, C_in = 512, 256, 384
+    x = synth.activations(T, C_in, seed=7, outlier_seed=8).float().numpy()
+    dy = synth.normal((T, C_out), 1e-3, 9).float().numpy()
+    qx, sx = oracle.quant_act_128x1(x, P2)
+    qdy, sdy = oracle.quant_act_128x1(dy, P2)
+    got = _run(qdy, sdy, qx, sx, C_in, gran=1)
+    ref, tol = oracle.gemm_full(qdy, sdy, qx, sx, sb_gran=1)
+    assert_gemm_close(got, ref, tol, False, "pow2 per-column")
+
+
+def test_pow2_gemm_long_k_against_software_promotion():
+    """K = 8192 (the Wgrad reduction length) with wide scale spread."""
+    M, N, K = 128, 256, 8192
+    qa, sa, qw, sw = _operands(M, N, K, seed=11)
+    got = _run(qa, sa, qw, sw, N)
+    ref, tol = oracle.gemm_full(qa, sa, qw, sw)
+    err = assert_gemm_close(got, ref, tol, False, "pow2 K=8192")
+    assert err < 1.0
+
+
+def test_pow2_gemm_reports_non_power_of_two_scale():
+    M, N, K = 128, 256, 256
+    qa, sa, qw, sw = _operands(M, N, K, seed=13)
+    sa = sa.copy()
+    sa[1, 5] = np.float32(0.75)
+    D = torch.empty((M, N), dtype=torch.float32, device=dev())
+    fg.fp8_blockscaled_gemm_pow2(to_dev(qa), to_dev(sa), to_dev(qw), to_dev(sw), D)
+    assert fg.fp8_get_status() == fg.FP8_ERR_VALUE
+    assert fg.fp8_get_status() == fg.FP8_OK
