@@ -88,9 +88,8 @@ struct MxParams {
 };
 
 struct __align__(8) MxShared {
-    uint64_t full[NS];
+    uint64_t full[NS];     // operands landed (TMA bytes) and scales stored (4 scale warps)
     uint64_t empty[NS];
-    uint64_t sf_full[NS];
     uint64_t acc_full;
     uint64_t acc_empty;
     uint64_t drain;
@@ -221,6 +220,12 @@ __device__ void mx_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, cons
     }
 }
 
+// The tensor core takes a new MMA only about when the previous one ends, so
+// the issuing thread runs at most one MMA ahead, and every cycle it spends on
+// anything else while the last queued MMA drains leaves the tensor core
+// idle.  The loop therefore waits for the next stage before issuing the
+// current stage's last MMA, so the barrier latency hides behind the MMAs
+// still executing, and it spins rather than suspends on barriers.
 __device__ void mx_mma(const MxParams& p, uint8_t* smem, MxShared& sh, int64_t nmb, int64_t nnb,
                        int64_t nkb)
 {
@@ -229,36 +234,40 @@ __device__ void mx_mma(const MxParams& p, uint8_t* smem, MxShared& sh, int64_t n
     const uint32_t b_base = a_base + NS * A_BYTES;
     const uint32_t sf_base = b_base + NS * B_BYTES;
     const uint32_t tmem = sh.tmem_base;
-    int64_t it = 0;
+    const int64_t ntiles = nmb * nnb;
+    uint32_t it = 0;          // K-blocks consumed so far (stage it % NS, round it / NS)
     uint32_t tcount = 0;
     bool ok = true;
-    for (int64_t tile = blockIdx.x; ok && tile < nmb * nnb; tile += gridDim.x, ++tcount) {
+    for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++tcount) {
         int64_t mb, nb;
         gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
         const int64_t n0 = nb * BN;
         const int64_t n_valid = (p.N - n0 < BN) ? (p.N - n0) : BN;
         const uint32_t idesc = idesc_mx_e4m3(BM, (uint32_t)n_valid, (uint32_t)p.b_major);
         // the epilogue has read the previous tile's accumulator
-        if (!mbar_wait(&sh.acc_empty, (tcount & 1u) ^ 1u, abort, p.timeout_ns)) break;
-        tc_fence_after();
+        ok = mbar_wait_spin(&sh.acc_empty, (tcount & 1u) ^ 1u, abort, p.timeout_ns) &&
+             mbar_wait_spin(&sh.full[it % NS], (it / NS) & 1u, abort, p.timeout_ns);
+        if (!ok) break;
         for (int64_t kb = 0; kb < nkb; ++kb, ++it) {
-            const int s = (int)(it % NS);
-            const uint32_t ph = (uint32_t)((it / NS) & 1);
-            if (!mbar_wait(&sh.sf_full[s], ph, abort, p.timeout_ns) ||
-                !mbar_wait(&sh.full[s], ph, abort, p.timeout_ns)) {
-                ok = false;
-                break;
-            }
+            const uint32_t s = it % NS;
             tc_fence_after();
             const uint32_t a_addr = a_base + s * A_BYTES;
             const uint32_t b_addr = b_base + s * B_BYTES;
             const uint32_t sf_addr = sf_base + s * SF_BYTES;
-            const uint32_t sfa = tmem + SF_COL0 + (uint32_t)s * SF_SLOT_COLS;
+            const uint32_t sfa = tmem + SF_COL0 + s * SF_SLOT_COLS;
             tmem_cp_32x128b_x4(sfa, sf_addr);                               // SFA, rows 0-127
             tmem_cp_32x128b_x4(sfa + SFB_OFF, sf_addr + SFA_BYTES);         // SFB, columns 0-127
             tmem_cp_32x128b_x4(sfa + SFB_OFF + 4, sf_addr + SFA_BYTES + 512);   // columns 128-255
 #pragma unroll
             for (int k = 0; k < BK / 32; ++k) {
+                if (k == BK / 32 - 1 && kb + 1 < nkb) {
+                    // next stage of this tile: wait while this stage's MMAs run
+                    const uint32_t nx = it + 1;
+                    if (!mbar_wait_spin(&sh.full[nx % NS], (nx / NS) & 1u, abort, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                }
                 const uint64_t adesc = smem_desc_sw128(a_addr + k * 32, 16, 1024);
                 const uint64_t bdesc = (p.b_major == FP8_B_KMAJOR)
                                            ? smem_desc_sw128(b_addr + k * 32, 16, 1024)
@@ -266,6 +275,7 @@ __device__ void mx_mma(const MxParams& p, uint8_t* smem, MxShared& sh, int64_t n
                 mma_mxf8(tmem, adesc, bdesc, idesc, sfa, sfa + SFB_OFF, (kb | k) ? 1u : 0u);
             }
             mma_commit(&sh.empty[s]);        // stage and scale slot free once these are done
+            if (!ok) break;
         }
         if (!ok) break;
         mma_commit(&sh.acc_full);            // the tile's sum is complete
@@ -348,7 +358,7 @@ __device__ void mx_scale_writer(const MxParams& p, uint8_t* smem, MxShared& sh, 
                         *reinterpret_cast<uint32_t*>(sf + off_b1) = wb1;
                         fence_proxy_async_smem();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(&sh.sf_full[s]);
+                        if (lane == 0) mbar_arrive(&sh.full[s]);
                     } else {
                         ok = false;
                     }
@@ -430,9 +440,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
-            mbar_init(&sh.full[s], 1);
+            mbar_init(&sh.full[s], 1 + NUM_SF_WARPS);
             mbar_init(&sh.empty[s], 1);
-            mbar_init(&sh.sf_full[s], NUM_SF_WARPS);
         }
         mbar_init(&sh.acc_full, 1);
         mbar_init(&sh.acc_empty, NUM_EPI_WARPS);
