@@ -378,19 +378,21 @@ __global__ void __launch_bounds__(kThr128x1, 6) k_quant_128x1(const Tin* __restr
 // that single rounding -- and the FP32 values are quantized in 128x1 groups
 // along tokens, exactly as k_quant_128x1 quantizes an FP32 input.
 //
-// CTA = 256 threads per tile of 128 tokens x 128 channels (one channel block,
-// hence one cached scale per token).  The 16 KB code tile is staged with
-// cp.async; warp w then owns tokens 16w .. 16w+15 and lane l channels
-// 4l .. 4l+3, read as one 32-bit word per token (a warp reads a whole
-// 128-byte row, conflict-free).  Pass 1: max-abs, combined over the 8 warps
-// through shared memory.  Pass 2: each thread encodes its 16 tokens of each
-// of its 4 channels into one 16-byte word.  The staged tile is dead by then,
-// so the transposed codes go back into the same shared memory (16-byte chunks
-// XOR-swizzled by (channel / 4) % 8, conflict-free) and leave as coalesced
-// 128-byte rows of qT.
-// Grid: x = C/128, y = T/128.
+// CTA = 256 threads over kReqTiles consecutive tiles of 128 tokens x 128
+// channels (one channel block, hence one cached scale per token), with the
+// next tile's 16 KB of codes and 128 scales loading (cp.async, double
+// buffered) while the current one is processed.  Per tile, warp w owns
+// tokens 16w .. 16w+15 and lane l channels 4l .. 4l+3, read as one 32-bit
+// word per token (a warp reads a whole 128-byte row, conflict-free).
+// Pass 1: max-abs, combined over the 8 warps through shared memory.  Pass 2:
+// each thread encodes its 16 tokens of each of its 4 channels into one
+// 16-byte word.  The staged tile is dead by then, so the transposed codes go
+// back into the same buffer (16-byte chunks XOR-swizzled by (channel / 4) %
+// 8, conflict-free) and leave as coalesced 128-byte rows of qT.
+// Grid: x = C/128, y = ceil(T/128 / kReqTiles).
 constexpr int kReqTok = 128;
 constexpr int kReqCh = 128;
+constexpr int kReqTiles = 4;
 
 __device__ __forceinline__ void decode4_e4m3(uint32_t w, float (&f)[4])
 {
@@ -401,93 +403,124 @@ __device__ __forceinline__ void decode4_e4m3(uint32_t w, float (&f)[4])
     f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
 }
 
-__global__ void __launch_bounds__(256) k_requant_128x1(const uint8_t* __restrict__ q, int64_t ldq,
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gsrc)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__global__ void __launch_bounds__(256, 4) k_requant_128x1(const uint8_t* __restrict__ q, int64_t ldq,
                                                        const float* __restrict__ sA, int64_t T,
                                                        int64_t C, uint8_t* __restrict__ qT,
                                                        int64_t ldqT, float* __restrict__ s, int mode)
 {
-    __shared__ __align__(16) uint8_t tile[kReqTok * kReqCh];      // codes, then transposed codes
+    __shared__ __align__(16) uint8_t tile[2][kReqTok * kReqCh];   // codes, then transposed codes
     __shared__ __align__(16) float part[8][kReqCh];
-    __shared__ float scl[kReqTok];
+    __shared__ float scl[2][kReqTok];
 
-    const int64_t tb = blockIdx.y;
     const int64_t cb = blockIdx.x;
-    const int64_t t0 = tb * kReqTok;
     const int64_t c0 = cb * kReqCh;
+    const int64_t ntb = T / kReqTok;
+    const int64_t tb0 = (int64_t)blockIdx.y * kReqTiles;
     const int w = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
+    auto stage = [&](int64_t tb, int buf) {
+        const int64_t t0 = tb * kReqTok;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int id = threadIdx.x + 256 * i;
-        const int r = id >> 3, j = id & 7;
-        cp_async16(&tile[r * kReqCh + j * 16], q + (t0 + r) * ldq + c0 + j * 16);
-    }
-    if (threadIdx.x < kReqTok) scl[threadIdx.x] = __ldg(sA + cb * T + t0 + threadIdx.x);
-    cp_async_wait_all();
-    __syncthreads();
+        for (int i = 0; i < 4; ++i) {
+            const int id = threadIdx.x + 256 * i;
+            const int r = id >> 3, j = id & 7;
+            cp_async16(&tile[buf][r * kReqCh + j * 16], q + (t0 + r) * ldq + c0 + j * 16);
+        }
+        if (threadIdx.x < kReqTok) cp_async4(&scl[buf][threadIdx.x], sA + cb * T + t0 + threadIdx.x);
+    };
 
-    // pass 1: max-abs of the dequantized values of channels 4l..4l+3
-    const uint32_t* tw = reinterpret_cast<const uint32_t*>(tile);
-    float a[4] = {0.f, 0.f, 0.f, 0.f};
+    stage(tb0, 0);
+    cp_async_commit();
+    for (int j = 0; j < kReqTiles; ++j) {
+        const int64_t tb = tb0 + j;
+        if (tb >= ntb) break;                          // block-uniform
+        const int buf = j & 1;
+        const bool more = j + 1 < kReqTiles && tb + 1 < ntb;
+        if (more) stage(tb + 1, buf ^ 1);              // its buffer was freed by tile j - 1
+        cp_async_commit();
+        cp_async_wait_group<1>();                      // tile j's group has landed
+        __syncthreads();
+
+        // pass 1: max-abs of the dequantized values of channels 4l..4l+3
+        const uint32_t* tw = reinterpret_cast<const uint32_t*>(tile[buf]);
+        const float* sc_t = scl[buf];
+        float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
-    for (int i = 0; i < 16; ++i) {
-        const int t = w * 16 + i;
-        float f[4];
-        decode4_e4m3(tw[t * (kReqCh / 4) + lane], f);
-        const float sc = scl[t];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) a[j] = fmaxf(a[j], fabsf(__fmul_rn(f[j], sc)));
-    }
-    *reinterpret_cast<float4*>(&part[w][4 * lane]) = make_float4(a[0], a[1], a[2], a[3]);
-    __syncthreads();
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const float4 p = *reinterpret_cast<const float4*>(&part[k][4 * lane]);
-        a[0] = fmaxf(a[0], p.x); a[1] = fmaxf(a[1], p.y);
-        a[2] = fmaxf(a[2], p.z); a[3] = fmaxf(a[3], p.w);
-    }
-    GroupScale g[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) g[j] = group_scale(a[j], mode);
-
-    // pass 2: encode 16 tokens x 4 channels into four 16-byte words
-    uint32_t out[4][4];
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-        float v[4][4];   // [token][channel]
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int t = w * 16 + q4 * 4 + u;
+        for (int i = 0; i < 16; ++i) {
+            const int t = w * 16 + i;
             float f[4];
             decode4_e4m3(tw[t * (kReqCh / 4) + lane], f);
-            const float sc = scl[t];
+            const float sc = sc_t[t];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) v[u][j] = __fmul_rn(f[j], sc);
+            for (int k = 0; k < 4; ++k) a[k] = fmaxf(a[k], fabsf(__fmul_rn(f[k], sc)));
         }
+        *reinterpret_cast<float4*>(&part[w][4 * lane]) = make_float4(a[0], a[1], a[2], a[3]);
+        __syncthreads();
 #pragma unroll
-        for (int j = 0; j < 4; ++j) out[j][q4] = encode4(v[0][j], v[1][j], v[2][j], v[3][j], g[j].inv);
-    }
-    __syncthreads();   // every read of the staged codes is done
+        for (int k = 0; k < 8; ++k) {
+            const float4 pv = *reinterpret_cast<const float4*>(&part[k][4 * lane]);
+            a[0] = fmaxf(a[0], pv.x); a[1] = fmaxf(a[1], pv.y);
+            a[2] = fmaxf(a[2], pv.z); a[3] = fmaxf(a[3], pv.w);
+        }
+        GroupScale g[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const int c = 4 * lane + j;
-        const int chunk = w ^ (lane & 7);
-        *reinterpret_cast<uint4*>(&tile[c * kReqTok + chunk * 16]) =
-            make_uint4(out[j][0], out[j][1], out[j][2], out[j][3]);
-    }
-    if (w == 0) {
+        for (int k = 0; k < 4; ++k) g[k] = group_scale(a[k], mode);
+
+        // pass 2: encode 16 tokens x 4 channels into four 16-byte words
+        uint32_t out[4][4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) s[tb * C + c0 + 4 * lane + j] = g[j].s;
-    }
-    __syncthreads();
+        for (int q4 = 0; q4 < 4; ++q4) {
+            float v[4][4];   // [token][channel]
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int id = threadIdx.x + 256 * i;
-        const int c = id >> 3, chunk = id & 7;
-        const uint4 v = *reinterpret_cast<const uint4*>(&tile[c * kReqTok + ((chunk ^ ((c >> 2) & 7)) * 16)]);
-        *reinterpret_cast<uint4*>(qT + (c0 + c) * ldqT + t0 + chunk * 16) = v;
+            for (int u = 0; u < 4; ++u) {
+                const int t = w * 16 + q4 * 4 + u;
+                float f[4];
+                decode4_e4m3(tw[t * (kReqCh / 4) + lane], f);
+                const float sc = sc_t[t];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) v[u][k] = __fmul_rn(f[k], sc);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) out[k][q4] = encode4(v[0][k], v[1][k], v[2][k], v[3][k], g[k].inv);
+        }
+        __syncthreads();   // every read of the staged codes and of part is done
+        uint8_t* tl = tile[buf];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int c = 4 * lane + k;
+            const int chunk = w ^ (lane & 7);
+            *reinterpret_cast<uint4*>(&tl[c * kReqTok + chunk * 16]) =
+                make_uint4(out[k][0], out[k][1], out[k][2], out[k][3]);
+        }
+        if (w == 0) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) s[tb * C + c0 + 4 * lane + k] = g[k].s;
+        }
+        __syncthreads();
+        const int64_t t0 = tb * kReqTok;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int id = threadIdx.x + 256 * i;
+            const int c = id >> 3, chunk = id & 7;
+            const uint4 v = *reinterpret_cast<const uint4*>(&tl[c * kReqTok + ((chunk ^ ((c >> 2) & 7)) * 16)]);
+            *reinterpret_cast<uint4*>(qT + (c0 + c) * ldqT + t0 + chunk * 16) = v;
+        }
+        __syncthreads();   // this buffer may be refilled by the next prefetch
     }
+    cp_async_wait_group<0>();
 }
 
 }  // namespace
@@ -525,7 +558,8 @@ cudaError_t launch_requant_128x1(const uint8_t* q, int64_t ldq, const float* sA,
                                  int64_t C, uint8_t* qT, int64_t ldqT, float* s, int mode,
                                  cudaStream_t st)
 {
-    const dim3 grid((unsigned)(C / kReqCh), (unsigned)(T / kReqTok));
+    const int64_t ntb = T / kReqTok;
+    const dim3 grid((unsigned)(C / kReqCh), (unsigned)((ntb + kReqTiles - 1) / kReqTiles));
     k_requant_128x1<<<grid, 256, 0, st>>>(q, ldq, sA, T, C, qT, ldqT, s, mode);
     return cudaGetLastError();
 }
