@@ -245,8 +245,9 @@ def describe(workload):
             # the forward pass's cache of X, made once outside the timed region
             qx, sx = fg.quant_act_1x128(wl["x"].to(d))
             return linear.WgradCachedStep(qx, sx, wl["dy"].to(d))
-    elif workload == "moe":
+    elif workload in ("moe", "moe_pow2_tc"):
         wl = synth.moe()
+        tc = workload == "moe_pow2_tc"
         lay = wl["layout"]
         topk = lay.topk.to(torch.int32)
         G, N, K = wl["w"].shape
@@ -254,7 +255,8 @@ def describe(workload):
         M = int(lay.counts.sum())
         desc = dict(workload="moe grouped fprop, 32 experts W_e[2048,7168], 16384 tokens "
                     "top-8 Zipf(1.1): 1x128 quantize tokens, FP8 dispatch to 128-padded "
-                    "groups, 128x128 quantize weights, grouped GEMM, bf16 out",
+                    "groups, 128x128 quantize weights, grouped GEMM, bf16 out"
+                    + (", pow2 scales applied in the tensor cores (UE8M0 block scaling)" if tc else ""),
                     M=M, N=N, K=K, M_padded=lay.m_total, tokens=T)
         inputs = [wl["x"], wl["w"], topk]
         # tokens read once (2 B) + codes written (1 B); dispatched codes read
@@ -263,6 +265,9 @@ def describe(workload):
                        + G * N * K * 3)
 
         def make(d):
+            if tc:
+                return linear.MoeStep(wl["x"].to(d), topk.to(d), wl["w"].to(d),
+                                      scale_mode=SCALE_POW2, tensor_core_scaling=True)
             return linear.MoeStep(wl["x"].to(d), topk.to(d), wl["w"].to(d))
     else:
         raise SystemExit(f"unknown workload {workload}")
@@ -290,7 +295,7 @@ def oracle_sample(workload, budget_s: float = 20.0, described=None):
     mode = SCALE_POW2 if "pow2" in workload else oracle.SCALE_FP32
     gemm_kw = {}
     t0 = time.perf_counter()
-    if workload in ("fprop", "fprop_pow2_tc", "pr1", "dgrad", "moe"):
+    if workload in ("fprop", "fprop_pow2_tc", "pr1", "dgrad", "moe", "moe_pow2_tc"):
         xa = wl["dy"] if workload == "dgrad" else wl["x"]
         w = wl["w"].reshape(-1, wl["w"].shape[-1])
         ra, rw = min(64, xa.shape[0]), min(256, w.shape[0])
@@ -348,7 +353,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="fprop",
                     choices=["fprop", "fprop_pow2_tc", "pr1", "dgrad", "wgrad", "wgrad_pow2",
-                             "wgrad_pow2_tc", "wgrad_cached", "moe"])
+                             "wgrad_pow2_tc", "wgrad_cached", "moe", "moe_pow2_tc"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -46,6 +46,7 @@ EXPORTED = (
     "fp8_set_wait_timeout_ns", "fp8_selftest_wait_timeout", "fp8_device_supported",
     "fp8_moe_dispatch_workspace_bytes", "fp8_moe_dispatch", "fp8_moe_combine",
     "fp8_moe_dispatch_noalloc", "fp8_requant_1x128_to_128x1", "fp8_blockscaled_gemm_pow2",
+    "fp8_grouped_gemm_pow2",
 )
 
 
@@ -79,6 +80,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fp8_blockscaled_gemm_pow2.argtypes = [_P, _P, _P, _I, _P, _I, _I64, _I64, _I64, _P, _I,
                                               _I64, _P]
     lib.fp8_blockscaled_gemm_pow2.restype = _I
+    lib.fp8_grouped_gemm_pow2.argtypes = [_P, _P, _P, _P, _P, _I, _I64, _I64, _I64, _P, _I, _P]
+    lib.fp8_grouped_gemm_pow2.restype = _I
     lib.fp8_grouped_gemm.argtypes = [_P, _P, _P, _P, _P, _I, _I64, _I64, _I64, _P, _I, _P]
     lib.fp8_grouped_gemm.restype = _I
     lib.fp8_get_status.argtypes = [_P]
@@ -204,6 +207,15 @@ def fp8_blockscaled_gemm_pow2(A, sA, B, sB, D, b_major: int = B_KMAJOR, sb_gran:
     _check(load_library().fp8_blockscaled_gemm_pow2(
         _ptr(A), _ptr(sA), _ptr(B), b_major, _ptr(sB), sb_gran, M, N, K, _ptr(D),
         _out_dtype(D), _row_stride(D), _stream(stream)), "fp8_blockscaled_gemm_pow2")
+
+
+def fp8_grouped_gemm_pow2(A, sA, B, sB, group_offsets, D, stream=None) -> None:
+    """fp8_grouped_gemm for power-of-two scales, scaled inside the tensor cores."""
+    M_total, K = A.shape
+    G, N, _ = B.shape
+    _check(load_library().fp8_grouped_gemm_pow2(
+        _ptr(A), _ptr(sA), _ptr(B), _ptr(sB), _ptr(group_offsets), G, M_total, N, K, _ptr(D),
+        _out_dtype(D), _stream(stream)), "fp8_grouped_gemm_pow2")
 
 
 def fp8_grouped_gemm(A, sA, B, sB, group_offsets, D, stream=None) -> None:

@@ -177,8 +177,28 @@ FP8FG_API int fp8_blockscaled_gemm_pow2(const uint8_t* A, const float* sA, const
         !aligned(sB, 4) || (ldd * osz) % 16)
         return FP8_ERR_ALIGN;
     if (!device_is_sm100()) return FP8_ERR_DEVICE;
-    return launch_blockscaled_gemm_mx(A, sA, B, b_major, sB, sb_gran, M, N, K, D, out_dtype, ldd,
-                                      static_cast<cudaStream_t>(stream));
+    return launch_blockscaled_gemm_mx(A, sA, B, b_major, sB, sb_gran, M, N, K, nullptr, 0, D,
+                                      out_dtype, ldd, static_cast<cudaStream_t>(stream));
+}
+
+FP8FG_API int fp8_grouped_gemm_pow2(const uint8_t* A, const float* sA, const uint8_t* B,
+                                    const float* sB, const int32_t* group_offsets, int G,
+                                    int64_t M_total, int64_t N, int64_t K, void* D, int out_dtype,
+                                    void* stream)
+{
+    if (!is_out(out_dtype)) return FP8_ERR_DTYPE;
+    if (G < 1 || G > 1024 || M_total < 0 || M_total > kMaxDim || M_total % 128 || N <= 0 ||
+        N > kMaxDim || N % 128 || K <= 0 || K > kMaxDim || K % 128 || (int64_t)G * N > kMaxDim)
+        return FP8_ERR_SHAPE;
+    if (M_total == 0) return FP8_OK;
+    if (!A || !sA || !B || !sB || !group_offsets || !D) return FP8_ERR_NULL;
+    const int osz = out_dtype == FP8_OUT_BF16 ? 2 : 4;
+    if (!aligned(A, 16) || !aligned(B, 16) || !aligned(D, 16) || !aligned(sA, 4) ||
+        !aligned(sB, 4) || !aligned(group_offsets, 4) || (N * osz) % 16)
+        return FP8_ERR_ALIGN;
+    if (!device_is_sm100()) return FP8_ERR_DEVICE;
+    return launch_blockscaled_gemm_mx(A, sA, B, FP8_B_KMAJOR, sB, 128, M_total, N, K, group_offsets,
+                                      G, D, out_dtype, N, static_cast<cudaStream_t>(stream));
 }
 
 FP8FG_API int fp8_grouped_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB,

@@ -324,6 +324,21 @@ __device__ __forceinline__ void gemm_tile_coord(int64_t tile, int64_t nmb, int64
     mb = mb0 + r % rows;
 }
 
+// Group of the 128-row block starting at row0: the largest e with
+// off[e] <= row0; -1 when row0 >= off[G] (rows outside every group).
+__device__ __forceinline__ int find_group(const int32_t* off, int G, int64_t row0)
+{
+    int lo = 0, hi = G;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if ((int64_t)off[mid] <= row0)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo < G ? lo : -1;
+}
+
 // Host: 2-D uint8 tensor map [outer][inner], rows `row_bytes` apart, boxes of
 // box_inner x box_outer bytes, 128-byte swizzle, zero fill out of bounds
 // (defined in gemm.cu; false when the driver's encoder is unavailable).

@@ -48,9 +48,11 @@ int read_and_clear_moe_status();
 
 // Power-of-two-scale GEMM on the tensor cores' UE8M0 block scaling
 // (gemm_mx.cu); same arguments as fp8_blockscaled_gemm.
+// fp8_grouped_gemm's layout when group_offsets is not null.
 int launch_blockscaled_gemm_mx(const uint8_t* A, const float* sA, const uint8_t* B, int b_major,
                                const float* sB, int sb_gran, int64_t M, int64_t N, int64_t K,
-                               void* D, int out_dtype, int64_t ldd, cudaStream_t st);
+                               const int32_t* group_offsets, int G, void* D, int out_dtype,
+                               int64_t ldd, cudaStream_t st);
 // Read and clear that module's status word (caller synchronised).
 int read_and_clear_mx_status();
 

@@ -73,20 +73,6 @@ struct GemmParams {
     uint64_t timeout_ns;
 };
 
-// Group of the 128-row block starting at row0: the largest e with
-// off[e] <= row0; -1 when row0 >= off[G] (rows outside every group).
-__device__ __forceinline__ int find_group(const int32_t* off, int G, int64_t row0)
-{
-    int lo = 0, hi = G;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if ((int64_t)off[mid] <= row0)
-            lo = mid;
-        else
-            hi = mid - 1;
-    }
-    return lo < G ? lo : -1;
-}
 
 struct __align__(16) Shared {
     float sbw[NUM_PROMO_WARPS][2][128];   // per-warp column scales (sb_gran == 1),

@@ -77,11 +77,15 @@ constexpr uint32_t SFB_BYTES = 1024;             // 256 columns x 4 bytes
 constexpr uint32_t SF_BYTES = SFA_BYTES + SFB_BYTES;
 constexpr uint32_t DYN_SMEM = 1024 + NS * (A_BYTES + B_BYTES + SF_BYTES);
 
+constexpr int MAX_GROUPS = 1024;
+
 struct MxParams {
     const float* sA;     // [K/128][M]
-    const float* sB;     // as for fp8_blockscaled_gemm
+    const float* sB;     // as for fp8_blockscaled_gemm / fp8_grouped_gemm
     void* D;
+    const int32_t* group_offsets;   // nullptr: dense
     int64_t M, N, K, ldd;
+    int G;
     int b_major, sb_gran, out_dtype;
     int b_box_rows;
     uint64_t timeout_ns;
@@ -95,6 +99,8 @@ struct __align__(8) MxShared {
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
+    int bad;
+    int32_t off[MAX_GROUPS + 1];   // grouped: the group offsets, validated on the device
 };
 
 // -------------------------------------------------------------- PTX helpers
@@ -187,9 +193,15 @@ __device__ void mx_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, cons
         int64_t mb, nb;
         gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
         const int64_t m0 = mb * BM, n0 = nb * BN;
+        int g = 0;
+        if (p.group_offsets) {
+            g = find_group(sh.off, p.G, m0);
+            if (g < 0) continue;
+        }
         const int64_t n_valid = (p.N - n0 < BN) ? (p.N - n0) : BN;
         const uint32_t b_bytes = (p.b_major == FP8_B_KMAJOR) ? (uint32_t)p.b_box_rows * BK
                                                              : (uint32_t)n_valid * BK;
+        const int32_t brow = (int32_t)((int64_t)g * p.N + n0);
         for (int64_t kb = 0; kb < nkb; ++kb) {
             const int s = (int)(it % NS);
             const uint32_t ph = (uint32_t)((it / NS) & 1);
@@ -203,7 +215,7 @@ __device__ void mx_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, cons
             uint8_t* b_dst = smem + NS * A_BYTES + s * B_BYTES;
             tma_load_2d(a_dst, tmA, &sh.full[s], (int32_t)(kb * BK), (int32_t)m0);
             if (p.b_major == FP8_B_KMAJOR) {
-                tma_load_2d(b_dst, tmB, &sh.full[s], (int32_t)(kb * BK), (int32_t)n0);
+                tma_load_2d(b_dst, tmB, &sh.full[s], (int32_t)(kb * BK), brow);
             } else {
                 tma_load_2d(b_dst, tmB, &sh.full[s], (int32_t)n0, (int32_t)(kb * BK));
                 if (n_valid > 128)
@@ -238,9 +250,10 @@ __device__ void mx_mma(const MxParams& p, uint8_t* smem, MxShared& sh, int64_t n
     uint32_t it = 0;          // K-blocks consumed so far (stage it % NS, round it / NS)
     uint32_t tcount = 0;
     bool ok = true;
-    for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++tcount) {
+    for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
         int64_t mb, nb;
         gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
+        if (p.group_offsets && find_group(sh.off, p.G, mb * BM) < 0) continue;
         const int64_t n0 = nb * BN;
         const int64_t n_valid = (p.N - n0 < BN) ? (p.N - n0) : BN;
         const uint32_t idesc = idesc_mx_e4m3(BM, (uint32_t)n_valid, (uint32_t)p.b_major);
@@ -279,6 +292,7 @@ __device__ void mx_mma(const MxParams& p, uint8_t* smem, MxShared& sh, int64_t n
         }
         if (!ok) break;
         mma_commit(&sh.acc_full);            // the tile's sum is complete
+        ++tcount;
     }
     mma_commit(&sh.drain);
     mbar_wait_drain(&sh.drain, 0, p.timeout_ns);
@@ -292,7 +306,7 @@ struct SfRegs {
     float b[2];
 };
 
-__device__ __forceinline__ void load_sf(const MxParams& p, int64_t m0, int64_t n0, int64_t kb,
+__device__ __forceinline__ void load_sf(const MxParams& p, int g, int64_t m0, int64_t n0, int64_t kb,
                                         int64_t nkb, int t, SfRegs& r)
 {
     const int64_t m = m0 + t;
@@ -305,8 +319,8 @@ __device__ __forceinline__ void load_sf(const MxParams& p, int64_t m0, int64_t n
         if (n < p.N) {
             if (p.sb_gran == 1)
                 v = __ldg(p.sB + kb * p.N + n);
-            else if (p.b_major == FP8_B_KMAJOR)
-                v = __ldg(p.sB + (n / 128) * nkb + kb);
+            else if (p.b_major == FP8_B_KMAJOR)   // grouped: sB [G][N/128][K/128]
+                v = __ldg(p.sB + ((int64_t)g * nnb128 + n / 128) * nkb + kb);
             else
                 v = __ldg(p.sB + kb * nnb128 + n / 128);
         }
@@ -333,11 +347,16 @@ __device__ void mx_scale_writer(const MxParams& p, uint8_t* smem, MxShared& sh, 
         int64_t mb, nb;
         gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
         const int64_t m0 = mb * BM, n0 = nb * BN;
+        int g = 0;
+        if (p.group_offsets) {
+            g = find_group(sh.off, p.G, m0);
+            if (g < 0) continue;
+        }
         // SF_AHEAD K-blocks of scale loads in flight per thread
         SfRegs ring[SF_AHEAD];
 #pragma unroll
         for (int u = 0; u < SF_AHEAD; ++u)
-            if (u < nkb) load_sf(p, m0, n0, u, nkb, t, ring[u]);
+            if (u < nkb) load_sf(p, g, m0, n0, u, nkb, t, ring[u]);
         for (int64_t kb0 = 0; ok && kb0 < nkb; kb0 += SF_AHEAD) {
 #pragma unroll
             for (int u = 0; u < SF_AHEAD; ++u) {
@@ -346,7 +365,7 @@ __device__ void mx_scale_writer(const MxParams& p, uint8_t* smem, MxShared& sh, 
                     const uint32_t wa = ue8m0_x4(ring[u].a, bad);
                     const uint32_t wb0 = ue8m0_x4(ring[u].b[0], bad);
                     const uint32_t wb1 = ue8m0_x4(ring[u].b[1], bad);
-                    if (kb + SF_AHEAD < nkb) load_sf(p, m0, n0, kb + SF_AHEAD, nkb, t, ring[u]);
+                    if (kb + SF_AHEAD < nkb) load_sf(p, g, m0, n0, kb + SF_AHEAD, nkb, t, ring[u]);
                     const int s = (int)(it % NS);
                     const uint32_t ph = (uint32_t)((it / NS) & 1);
                     // the copies and MMAs that last read this stage have completed
@@ -379,14 +398,16 @@ __device__ void mx_epilogue(const MxParams& p, MxShared& sh, int64_t nmb, int64_
     const int row = q * 32 + lane;
     const uint32_t taddr0 = sh.tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)col0;
     uint32_t tcount = 0;
-    for (int64_t tile = blockIdx.x; tile < nmb * nnb; tile += gridDim.x, ++tcount) {
+    for (int64_t tile = blockIdx.x; tile < nmb * nnb; tile += gridDim.x) {
         int64_t mb, nb;
         gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
+        if (p.group_offsets && find_group(sh.off, p.G, mb * BM) < 0) continue;
+        const uint32_t tph = tcount++ & 1u;
         const int64_t m = mb * BM + row;
         const int64_t n0 = nb * BN + col0;
         const bool active = n0 < p.N;           // warp-uniform
         const bool row_ok = m < p.M;
-        if (!warp_wait(&sh.acc_full, tcount & 1u, abort, p.timeout_ns, lane)) break;
+        if (!warp_wait(&sh.acc_full, tph, abort, p.timeout_ns, lane)) break;
         tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
@@ -447,6 +468,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_init(&sh.acc_empty, NUM_EPI_WARPS);
         mbar_init(&sh.drain, 1);
         sh.abort = 0;
+        sh.bad = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
@@ -455,11 +477,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_alloc(&sh.tmem_base, TMEM_COLS);
         tmem_relinquish();
     }
+    if (p.group_offsets)
+        for (int i = threadIdx.x; i <= p.G; i += NUM_THREADS) sh.off[i] = p.group_offsets[i];
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (threadIdx.x == 0) {
+        bool bad = false;
+        if (p.group_offsets) {
+            bad = sh.off[0] != 0 || (int64_t)sh.off[p.G] > p.M;
+            for (int e = 0; e < p.G; ++e) bad = bad || sh.off[e + 1] < sh.off[e] || (sh.off[e + 1] & 127);
+            if (bad && blockIdx.x == 0) report_error(FP8_ERR_SHAPE);
+        }
+        sh.bad = bad ? 1 : 0;
+    }
+    __syncthreads();
 
-    if (warp == 0) {
+    if (sh.bad) {
+        // malformed offsets: nothing is loaded, multiplied or written
+    } else if (warp == 0) {
         if (lane == 0) mx_producer(&tmA, &tmB, p, smem, sh, nmb, nnb, nkb);
         __syncwarp();
     } else if (warp == 1) {
@@ -496,26 +532,32 @@ bool ensure_mx_smem_attr()
 
 int launch_blockscaled_gemm_mx(const uint8_t* A, const float* sA, const uint8_t* B, int b_major,
                                const float* sB, int sb_gran, int64_t M, int64_t N, int64_t K,
-                               void* D, int out_dtype, int64_t ldd, cudaStream_t st)
+                               const int32_t* group_offsets, int G, void* D, int out_dtype,
+                               int64_t ldd, cudaStream_t st)
 {
     if (M == 0) return FP8_OK;
     CUtensorMap tmA, tmB;
     const int b_box_rows = N >= BN ? BN : (int)N;
     if (!make_map(&tmA, A, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, BM)) return FP8_ERR_LAUNCH;
-    const bool okB = (b_major == FP8_B_KMAJOR)
-                         ? make_map(&tmB, B, (uint64_t)K, (uint64_t)N, (uint64_t)K, BK,
-                                    (uint32_t)b_box_rows)
-                         : make_map(&tmB, B, (uint64_t)N, (uint64_t)K, (uint64_t)N, 128, BK);
+    bool okB;
+    if (b_major == FP8_B_KMAJOR) {
+        const uint64_t rows = (uint64_t)N * (uint64_t)(group_offsets ? G : 1);
+        okB = make_map(&tmB, B, (uint64_t)K, rows, (uint64_t)K, BK, (uint32_t)b_box_rows);
+    } else {
+        okB = make_map(&tmB, B, (uint64_t)N, (uint64_t)K, (uint64_t)N, 128, BK);
+    }
     if (!okB || !ensure_mx_smem_attr()) return FP8_ERR_LAUNCH;
 
     MxParams p;
     p.sA = sA;
     p.sB = sB;
     p.D = D;
+    p.group_offsets = group_offsets;
     p.M = M;
     p.N = N;
     p.K = K;
     p.ldd = ldd;
+    p.G = group_offsets ? G : 0;
     p.b_major = b_major;
     p.sb_gran = sb_gran;
     p.out_dtype = out_dtype;

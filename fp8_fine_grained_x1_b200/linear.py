@@ -32,7 +32,7 @@ from __future__ import annotations
 import torch
 
 from . import (B_KMAJOR, B_MNMAJOR, SCALE_FP32, SCALE_POW2, fp8_blockscaled_gemm,
-               fp8_blockscaled_gemm_pow2, fp8_grouped_gemm,
+               fp8_blockscaled_gemm_pow2, fp8_grouped_gemm, fp8_grouped_gemm_pow2,
                fp8_moe_combine, fp8_moe_dispatch, fp8_moe_dispatch_workspace_bytes,
                fp8_quant_act_128x1, fp8_quant_act_1x128, fp8_quant_w_128x128,
                fp8_requant_1x128_to_128x1, moe_capacity)
@@ -184,10 +184,14 @@ class MoeStep:
     weighted return to token order."""
     kernel_calls = 7      # quantize X, 4 dispatch kernels, quantize W, grouped GEMM (+1 memset)
 
-    def __init__(self, x, topk, w, out_dtype=torch.bfloat16, scale_mode=SCALE_FP32):
+    def __init__(self, x, topk, w, out_dtype=torch.bfloat16, scale_mode=SCALE_FP32,
+                 tensor_core_scaling=False):
         T, K = x.shape
         G, N, K2 = w.shape
         assert K == K2
+        if tensor_core_scaling and scale_mode != SCALE_POW2:
+            raise ValueError("tensor-core scaling needs power-of-two scales (SCALE_POW2)")
+        self._gemm = fp8_grouped_gemm_pow2 if tensor_core_scaling else fp8_grouped_gemm
         k = topk.shape[1]
         d = x.device
         self.x, self.topk, self.w, self.mode, self.G = x, topk, w, scale_mode, G
@@ -215,7 +219,7 @@ class MoeStep:
                             self.sw.view(G * N // 128, K // 128), self.mode, stream)
 
     def gemm(self, stream=None):
-        fp8_grouped_gemm(self.qa, self.sa, self.qw, self.sw, self.offsets, self.y, stream)
+        self._gemm(self.qa, self.sa, self.qw, self.sw, self.offsets, self.y, stream)
 
     def combine(self, weights, stream=None):
         T = self.x.shape[0]

@@ -190,6 +190,17 @@ int fp8_blockscaled_gemm_pow2(const uint8_t* A, const float* sA, const uint8_t* 
                               void* D, int out_dtype, int64_t ldd, void* stream);
 
 /*
+ * fp8_grouped_gemm for power-of-two scales, scaled inside the tensor cores
+ * as fp8_blockscaled_gemm_pow2 does ([P1] power-of-2 scales; [P5] the MoE
+ * part reads one expert's weights per group).  Arguments, layouts, sizes and
+ * errors as fp8_grouped_gemm; every sA / sB value must be 2^e with
+ * -126 <= e <= 127, else FP8_ERR_VALUE through the status word.
+ */
+int fp8_grouped_gemm_pow2(const uint8_t* A, const float* sA, const uint8_t* B, const float* sB,
+                          const int32_t* group_offsets, int G, int64_t M_total, int64_t N, int64_t K,
+                          void* D, int out_dtype, void* stream);
+
+/*
  * Grouped (MoE expert) block-scaled GEMM: rows [off[e], off[e+1]) of A are
  * multiplied by expert e's weight ([P4] MoE layer; [P5] each group only
  * loads the parameters of one expert).

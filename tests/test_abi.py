@@ -154,8 +154,9 @@ def test_requant_validation(lib):
     assert rq() in (fg.FP8_ERR_DEVICE, fg.FP8_OK)
 
 
-def test_grouped_validation(lib):
-    f = lib.fp8_grouped_gemm
+@pytest.mark.parametrize("name", ["fp8_grouped_gemm", "fp8_grouped_gemm_pow2"])
+def test_grouped_validation(lib, name):
+    f = getattr(lib, name)
     args = dict(A=FAKE, sA=FAKE2, B=FAKE3, sB=FAKE4, off=FAKE5, G=4, M=512, N=256, K=256,
                 D=0x60000, od=0)
 

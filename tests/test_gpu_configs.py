@@ -153,12 +153,15 @@ def test_wgrad_from_cached_fp8_activations():
     assert_gemm_close(d2h(dw)[pts[:, 0], pts[:, 1]], ref, tol, False, "wgrad from cache")
 
 
-def test_moe_grouped_fprop():
+@pytest.mark.parametrize("pow2_tc", [False, True], ids=["fp32_scales", "pow2_tensor_cores"])
+def test_moe_grouped_fprop(pow2_tc):
     wl = synth.moe()
     lay = wl["layout"]
     G, N, K = wl["w"].shape
+    mode = fg.SCALE_POW2 if pow2_tc else fg.SCALE_FP32
     topk = lay.topk.to(torch.int32)
-    step = linear.MoeStep(wl["x"].to(dev()), topk.to(dev()), wl["w"].to(dev()))
+    step = linear.MoeStep(wl["x"].to(dev()), topk.to(dev()), wl["w"].to(dev()), scale_mode=mode,
+                          tensor_core_scaling=pow2_tc)
     y = step()
     torch.cuda.synchronize()
     assert fg.fp8_get_status() == fg.FP8_OK
@@ -168,9 +171,9 @@ def test_moe_grouped_fprop():
     assert np.array_equal(step.row_token.cpu().numpy()[:lay.m_total], lay.row_token.numpy())
 
     # tokens and weights quantized by the oracle, bit-exact
-    qx, sx = oracle.quant_act_1x128(_bits(wl["x"]))
+    qx, sx = oracle.quant_act_1x128(_bits(wl["x"]), mode)
     assert np.array_equal(step.qx.cpu().numpy(), qx) and np.array_equal(step.sx.cpu().numpy(), sx)
-    qw, sw = oracle.quant_w_128x128(_bits(wl["w"].view(G * N, K)))
+    qw, sw = oracle.quant_w_128x128(_bits(wl["w"].view(G * N, K)), mode)
     assert np.array_equal(step.qw.cpu().numpy().reshape(G * N, K), qw)
     assert np.array_equal(step.sw.cpu().numpy().reshape(G * N // 128, K // 128), sw)
     qw = qw.reshape(G, N, K)

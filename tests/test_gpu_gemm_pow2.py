@@ -87,3 +87,50 @@ def test_pow2_gemm_reports_non_power_of_two_scale():
     fg.fp8_blockscaled_gemm_pow2(to_dev(qa), to_dev(sa), to_dev(qw), to_dev(sw), D)
     assert fg.fp8_get_status() == fg.FP8_ERR_VALUE
     assert fg.fp8_get_status() == fg.FP8_OK
+
+
+def _pow2(s):
+    """Nearest power of two of each positive scale (test input construction)."""
+    return np.exp2(np.round(np.log2(s))).astype(np.float32)
+
+
+def _grouped_pow2_operands(counts, N, K, seed):
+    G = len(counts)
+    off = np.zeros(G + 1, np.int32)
+    off[1:] = np.cumsum([(c + 127) // 128 * 128 for c in counts])
+    A = np.zeros((int(off[-1]), K), np.uint8)
+    for e, c in enumerate(counts):
+        A[off[e]:off[e] + c] = synth.random_e4m3_codes((c, K), seed + e)
+    sA = _pow2(synth.random_scales((K // 128, A.shape[0]), seed + 100))
+    B = synth.random_e4m3_codes((G, N, K), seed + 200)
+    sB = _pow2(synth.random_scales((G, N // 128, K // 128), seed + 300))
+    return A, sA, B, sB, off
+
+
+@pytest.mark.parametrize("out", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("counts,N,K", [([130, 0, 5, 256], 256, 512), ([1, 300, 0, 0, 77], 384, 256)])
+def test_pow2_grouped_matches_oracle(counts, N, K, out):
+    A, sA, B, sB, off = _grouped_pow2_operands(counts, N, K, seed=len(counts) * 17 + N)
+    M_total = A.shape[0] + 128                                # one block beyond off[G]
+    A = np.concatenate([A, synth.random_e4m3_codes((128, K), 71)])
+    sA = np.ascontiguousarray(np.concatenate([sA, np.ones((K // 128, 128), np.float32)], axis=1))
+    D = torch.full((M_total, N), -3.0, dtype=out, device=dev())
+    fg.fp8_grouped_gemm_pow2(to_dev(A), to_dev(sA), to_dev(B), to_dev(sB), to_dev(off), D)
+    assert fg.fp8_get_status() == fg.FP8_OK
+    got = d2h(D)
+    pts = np.array([(m, n) for m in range(M_total) for n in range(N)], np.int64)
+    ref, tol, grp = oracle.grouped_gemm_points(A, sA, B, sB, off, pts)
+    inside = grp >= 0
+    assert_gemm_close(got.reshape(-1)[inside], ref[inside], tol[inside], out == torch.bfloat16,
+                      "pow2 grouped")
+    assert np.all(got.reshape(-1)[~inside] == -3.0)           # rows beyond off[G] untouched
+
+
+def test_pow2_grouped_bad_offsets_report_shape_error_and_write_nothing():
+    A, sA, B, sB, off = _grouped_pow2_operands([128, 128], 256, 256, seed=5)
+    bad = off.copy()
+    bad[1] = 100                                              # not a multiple of 128
+    D = torch.full((A.shape[0], 256), 5.0, dtype=torch.float32, device=dev())
+    fg.fp8_grouped_gemm_pow2(to_dev(A), to_dev(sA), to_dev(B), to_dev(sB), to_dev(bad), D)
+    assert fg.fp8_get_status() == fg.FP8_ERR_SHAPE
+    assert torch.all(D == 5.0)
