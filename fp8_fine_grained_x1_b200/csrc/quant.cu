@@ -241,6 +241,7 @@ __global__ void __launch_bounds__(256) k_quant_w128(const Tin* __restrict__ w, i
 
 constexpr int kTok = 128;        // tokens per tile (one group along tokens)
 constexpr int kThr128x1 = 256;
+constexpr int kTiles128x1 = 4;   // token blocks per CTA, double-buffered
 // Tile geometry per input type: 128-byte row segments (64 BF16 or 32 FP32
 // channels), threads own channel pairs x (kTok / kGroups) tokens.  (256-byte
 // segments with 512 threads measured slower.)
@@ -263,7 +264,10 @@ struct Geo128x1 {
 // a first pass takes the max-abs, the token groups combine theirs through
 // shared memory, and a second pass encodes the thread's tokens of each
 // channel into one 16- or 8-byte store per channel of the transposed output.
-// Grid: x = ceil(C / kCh), y = T/128.
+// Each CTA walks kTiles128x1 consecutive token blocks of its channel
+// slice, loading the next block (cp.async, double buffered) while it
+// processes the current one.
+// Grid: x = ceil(C / kCh), y = ceil(T/128 / kTiles128x1).
 template <typename Tin>
 struct Pair;
 template <>
@@ -289,85 +293,129 @@ __device__ __forceinline__ void cp_async_wait_all()
 {
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gsrc)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 
 template <typename Tin>
-__global__ void __launch_bounds__(kThr128x1, 6) k_quant_128x1(const Tin* __restrict__ x, int64_t C,
-                                                              int64_t ldx, uint8_t* __restrict__ qT,
-                                                              int64_t ldqT, float* __restrict__ s, int mode)
+__global__ void __launch_bounds__(kThr128x1, 5) k_quant_128x1(const Tin* __restrict__ x, int64_t ntb,
+                                                              int64_t C, int64_t ldx,
+                                                              uint8_t* __restrict__ qT, int64_t ldqT,
+                                                              float* __restrict__ s, int mode)
 {
     using G = Geo128x1<Tin>;
     constexpr int kElemsPerChunk = 16 / (int)sizeof(Tin);
     constexpr int kChunksPerRow = G::kCh / kElemsPerChunk;           // 8
     constexpr int kChunksPerThread = kTok * kChunksPerRow / kThr128x1;   // 4
-    __shared__ __align__(16) Tin tile[kTok][G::kCh];
+    __shared__ __align__(16) Tin tile[2][kTok][G::kCh];
     __shared__ float2 part[G::kGroups][G::kPairs];
+    // transposed codes of one token block: kCh rows of 128 bytes, 16-byte
+    // chunks XOR-swizzled by row so both the scattered writes and the row
+    // reads are conflict-free
+    __shared__ __align__(16) uint8_t outT[G::kCh][kTok];
 
-    const int64_t tb = blockIdx.y;
     const int64_t c0 = (int64_t)blockIdx.x * G::kCh;
+    const int64_t tb0 = (int64_t)blockIdx.y * kTiles128x1;
+    const int64_t tb_end = ntb < tb0 + kTiles128x1 ? ntb : tb0 + kTiles128x1;
 
-    // 1. stage the tile (channels beyond C are zero; C % 8 == 0)
+    // stage token block tb into buffer buf (channels beyond C are zero; C % 8 == 0)
+    auto stage = [&](int64_t tb, int buf) {
 #pragma unroll
-    for (int i = 0; i < kChunksPerThread; ++i) {
-        const int id = threadIdx.x + kThr128x1 * i;
-        const int r = id / kChunksPerRow;
-        const int j = id % kChunksPerRow;
-        const int64_t ch = c0 + j * kElemsPerChunk;
-        if (ch < C)
-            cp_async16(&tile[r][j * kElemsPerChunk], x + (tb * kTok + r) * ldx + ch);
-        else
-            *reinterpret_cast<uint4*>(&tile[r][j * kElemsPerChunk]) = make_uint4(0, 0, 0, 0);
-    }
-    cp_async_wait_all();
-    __syncthreads();
+        for (int i = 0; i < kChunksPerThread; ++i) {
+            const int id = threadIdx.x + kThr128x1 * i;
+            const int r = id / kChunksPerRow;
+            const int j = id % kChunksPerRow;
+            const int64_t ch = c0 + j * kElemsPerChunk;
+            if (ch < C)
+                cp_async16(&tile[buf][r][j * kElemsPerChunk], x + (tb * kTok + r) * ldx + ch);
+            else
+                *reinterpret_cast<uint4*>(&tile[buf][r][j * kElemsPerChunk]) = make_uint4(0, 0, 0, 0);
+        }
+    };
 
-    // 2. max-abs of channels 2p, 2p+1 over this thread's tokens, then over groups
     const int pch = threadIdx.x % G::kPairs;
     const int g = threadIdx.x / G::kPairs;
     const int t0 = g * G::kTokPerThr;
-    float a0 = 0.0f, a1 = 0.0f;
-#pragma unroll
-    for (int t = 0; t < G::kTokPerThr; ++t) {
-        const float2 v = Pair<Tin>::get(&tile[t0 + t][2 * pch]);
-        a0 = fmaxf(a0, fabsf(v.x));
-        a1 = fmaxf(a1, fabsf(v.y));
-    }
-    part[g][pch] = make_float2(a0, a1);
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < G::kGroups; ++i) {
-        const float2 q = part[i][pch];
-        a0 = fmaxf(a0, q.x);
-        a1 = fmaxf(a1, q.y);
-    }
-    const GroupScale g0 = group_scale(a0, mode);
-    const GroupScale g1 = group_scale(a1, mode);
-
-    // 3. encode this thread's tokens of each channel, store transposed
     const int64_t ch = c0 + 2 * pch;
-    if (ch < C) {   // C % 8 == 0: ch < C implies ch + 1 < C
-        uint32_t w0[G::kTokPerThr / 4], w1[G::kTokPerThr / 4];
+
+    stage(tb0, 0);
+    cp_async_commit();
+    for (int jt = 0; jt < kTiles128x1; ++jt) {
+        const int64_t tb = tb0 + jt;
+        if (tb >= tb_end) break;                       // block-uniform
+        const int buf = jt & 1;
+        if (tb + 1 < tb_end) stage(tb + 1, buf ^ 1);   // its buffer was freed by tile jt - 1
+        cp_async_commit();
+        cp_async_wait_group<1>();                      // tile jt has landed
+        __syncthreads();
+
+        // max-abs of channels 2p, 2p+1 over this thread's tokens, then over groups
+        float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
-        for (int q4 = 0; q4 < G::kTokPerThr / 4; ++q4) {
-            float2 v[4];
+        for (int t = 0; t < G::kTokPerThr; ++t) {
+            const float2 v = Pair<Tin>::get(&tile[buf][t0 + t][2 * pch]);
+            a0 = fmaxf(a0, fabsf(v.x));
+            a1 = fmaxf(a1, fabsf(v.y));
+        }
+        part[g][pch] = make_float2(a0, a1);
+        __syncthreads();
 #pragma unroll
-            for (int t = 0; t < 4; ++t) v[t] = Pair<Tin>::get(&tile[t0 + q4 * 4 + t][2 * pch]);
-            w0[q4] = encode4(v[0].x, v[1].x, v[2].x, v[3].x, g0.inv);
-            w1[q4] = encode4(v[0].y, v[1].y, v[2].y, v[3].y, g1.inv);
+        for (int i = 0; i < G::kGroups; ++i) {
+            const float2 q = part[i][pch];
+            a0 = fmaxf(a0, q.x);
+            a1 = fmaxf(a1, q.y);
         }
-        uint8_t* d0 = qT + ch * ldqT + tb * kTok + t0;
-        uint8_t* d1 = d0 + ldqT;
-        if constexpr (G::kTokPerThr == 16) {
-            *reinterpret_cast<uint4*>(d0) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
-            *reinterpret_cast<uint4*>(d1) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
-        } else {
-            *reinterpret_cast<uint2*>(d0) = make_uint2(w0[0], w0[1]);
-            *reinterpret_cast<uint2*>(d1) = make_uint2(w1[0], w1[1]);
+        const GroupScale g0 = group_scale(a0, mode);
+        const GroupScale g1 = group_scale(a1, mode);
+
+        // encode this thread's tokens of channels 2p, 2p+1 into the transposed
+        // tile (byte offset t0 of rows 2p and 2p+1, chunk-swizzled)
+        {
+            uint32_t w0[G::kTokPerThr / 4], w1[G::kTokPerThr / 4];
+#pragma unroll
+            for (int q4 = 0; q4 < G::kTokPerThr / 4; ++q4) {
+                float2 v[4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) v[t] = Pair<Tin>::get(&tile[buf][t0 + q4 * 4 + t][2 * pch]);
+                w0[q4] = encode4(v[0].x, v[1].x, v[2].x, v[3].x, g0.inv);
+                w1[q4] = encode4(v[0].y, v[1].y, v[2].y, v[3].y, g1.inv);
+            }
+            const int r0 = 2 * pch, r1 = 2 * pch + 1;
+            const int off0 = (t0 ^ ((r0 & 7) << 4)), off1 = (t0 ^ ((r1 & 7) << 4));
+            if constexpr (G::kTokPerThr == 16) {
+                *reinterpret_cast<uint4*>(&outT[r0][off0]) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+                *reinterpret_cast<uint4*>(&outT[r1][off1]) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+            } else {
+                *reinterpret_cast<uint2*>(&outT[r0][off0]) = make_uint2(w0[0], w0[1]);
+                *reinterpret_cast<uint2*>(&outT[r1][off1]) = make_uint2(w1[0], w1[1]);
+            }
+            if (g == 0 && ch < C) {   // s is only guaranteed 4-byte aligned: two scalar stores
+                s[tb * C + ch] = g0.s;
+                s[tb * C + ch + 1] = g1.s;
+            }
         }
-        if (g == 0) {   // s is only guaranteed 4-byte aligned: two scalar stores
-            s[tb * C + ch] = g0.s;
-            s[tb * C + ch + 1] = g1.s;
+        __syncthreads();
+        // whole 128-byte rows of qT: 8 threads per row, 16 bytes each
+        for (int id = threadIdx.x; id < G::kCh * 8; id += kThr128x1) {
+            const int r = id >> 3, c16 = id & 7;
+            const int64_t chr = c0 + r;
+            if (chr < C) {
+                const uint4 v = *reinterpret_cast<const uint4*>(&outT[r][(c16 << 4) ^ ((r & 7) << 4)]);
+                *reinterpret_cast<uint4*>(qT + chr * ldqT + tb * kTok + (c16 << 4)) = v;
+            }
         }
+        __syncthreads();   // the buffers may be rewritten by the next tile
     }
+    cp_async_wait_group<0>();
 }
 
 // ------------------------------------------------------------ requantize 1x128 -> 128x1
@@ -401,18 +449,6 @@ __device__ __forceinline__ void decode4_e4m3(uint32_t w, float (&f)[4])
     const float2 a = __half22float2(__half2(lo));
     const float2 b = __half22float2(__half2(hi));
     f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
-}
-
-__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gsrc)
-{
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group()
-{
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __global__ void __launch_bounds__(256, 4) k_requant_128x1(const uint8_t* __restrict__ q, int64_t ldq,
@@ -544,13 +580,15 @@ cudaError_t launch_quant_act_128x1(const void* x, int in_dtype, int64_t T, int64
                                    uint8_t* qT, int64_t ldqT, float* s, int mode, cudaStream_t st)
 {
     const int ch_tile = in_dtype == FP8_IN_BF16 ? Geo128x1<__nv_bfloat16>::kCh : Geo128x1<float>::kCh;
-    const dim3 grid((unsigned)((C + ch_tile - 1) / ch_tile), (unsigned)(T / kTok));
+    const int64_t ntb = T / kTok;
+    const dim3 grid((unsigned)((C + ch_tile - 1) / ch_tile),
+                    (unsigned)((ntb + kTiles128x1 - 1) / kTiles128x1));
     if (in_dtype == FP8_IN_BF16)
         k_quant_128x1<__nv_bfloat16><<<grid, kThr128x1, 0, st>>>(
-            static_cast<const __nv_bfloat16*>(x), C, ldx, qT, ldqT, s, mode);
+            static_cast<const __nv_bfloat16*>(x), ntb, C, ldx, qT, ldqT, s, mode);
     else
-        k_quant_128x1<float><<<grid, kThr128x1, 0, st>>>(static_cast<const float*>(x), C, ldx, qT,
-                                                   ldqT, s, mode);
+        k_quant_128x1<float><<<grid, kThr128x1, 0, st>>>(static_cast<const float*>(x), ntb, C, ldx,
+                                                         qT, ldqT, s, mode);
     return cudaGetLastError();
 }
 
