@@ -344,6 +344,25 @@ def oracle_sample(workload, budget_s: float = 20.0, described=None):
                 step_s=step_s)
 
 
+# ---------------------------------------------------------------- ranks
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The largest per-rank value over all ranks: each replica's time counts,
+    so the job's time is the slowest rank's (NCCL on the GPU, gloo on CPU)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, flops_per_step: float, ms_per_step: float) -> float:
+    """Whole-job TFLOP/s: every rank processes one step's work per step time."""
+    return world * flops_per_step / (ms_per_step * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------- main
 
 def main():
@@ -447,16 +466,13 @@ def main():
     quant_ms = sorted(ev_q0[i].elapsed_time(ev_g0[i]) for i in range(args.steps))
     gemm_avg = sum(gemm_ms) / len(gemm_ms)
     quant_avg = sum(quant_ms) / len(quant_ms)
-    if world > 1:
-        t = torch.tensor([ms_total], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, world, device)
     status = fg.fp8_get_status()
     if status != fg.FP8_OK:
         raise SystemExit(f"device status after timing: {fg.status_string(status)}")
 
     ms_per_step = ms_total / args.steps
-    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    value = job_throughput(world, flops, ms_per_step)
     peaks = measured_peaks()
     # The GEMM is timed inside a long run of back-to-back steps: compare it
     # with the sustained (power-capped) BF16 peak x 2 (FP8 : BF16 = 2 : 1).
@@ -490,11 +506,8 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         e_ms = e0.elapsed_time(e1) / args.e2e_steps
-        if world > 1:
-            t = torch.tensor([e_ms], device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e_ms = max_over_ranks(e_ms, world, device)
+        e2e = {"value": job_throughput(world, flops, e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
 
     cpu = None
