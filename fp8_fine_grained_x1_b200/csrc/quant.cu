@@ -432,9 +432,10 @@ __global__ void __launch_bounds__(kThr128x1, 5) k_quant_128x1(const Tin* __restr
 // buffered) while the current one is processed.  Per tile, warp w owns
 // tokens 16w .. 16w+15 and lane l channels 4l .. 4l+3, read as one 32-bit
 // word per token (a warp reads a whole 128-byte row, conflict-free).
-// Pass 1: max-abs, combined over the 8 warps through shared memory.  Pass 2:
-// each thread encodes its 16 tokens of each of its 4 channels into one
-// 16-byte word.  The staged tile is dead by then, so the transposed codes go
+// Pass 1: dequantize once (the 64 products stay in registers) and take the
+// max-abs, combined over the 8 warps through shared memory.  Pass 2: each
+// thread encodes its 16 tokens of each of its 4 channels into one 16-byte
+// word.  The staged tile is dead by then, so the transposed codes go
 // back into the same buffer (16-byte chunks XOR-swizzled by (channel / 4) %
 // 8, conflict-free) and leave as coalesced 128-byte rows of qT.
 // Grid: x = C/128, y = ceil(T/128 / kReqTiles).
@@ -451,7 +452,7 @@ __device__ __forceinline__ void decode4_e4m3(uint32_t w, float (&f)[4])
     f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
 }
 
-__global__ void __launch_bounds__(256, 4) k_requant_128x1(const uint8_t* __restrict__ q, int64_t ldq,
+__global__ void __launch_bounds__(256, 3) k_requant_128x1(const uint8_t* __restrict__ q, int64_t ldq,
                                                        const float* __restrict__ sA, int64_t T,
                                                        int64_t C, uint8_t* __restrict__ qT,
                                                        int64_t ldqT, float* __restrict__ s, int mode)
@@ -490,18 +491,23 @@ __global__ void __launch_bounds__(256, 4) k_requant_128x1(const uint8_t* __restr
         cp_async_wait_group<1>();                      // tile j's group has landed
         __syncthreads();
 
-        // pass 1: max-abs of the dequantized values of channels 4l..4l+3
+        // pass 1: dequantize this thread's 16 tokens x 4 channels once (kept in
+        // registers for pass 2) and take their max-abs per channel
         const uint32_t* tw = reinterpret_cast<const uint32_t*>(tile[buf]);
         const float* sc_t = scl[buf];
+        float v[16][4];
         float a[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
+#pragma unroll
         for (int i = 0; i < 16; ++i) {
             const int t = w * 16 + i;
             float f[4];
             decode4_e4m3(tw[t * (kReqCh / 4) + lane], f);
             const float sc = sc_t[t];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) a[k] = fmaxf(a[k], fabsf(__fmul_rn(f[k], sc)));
+            for (int k = 0; k < 4; ++k) {
+                v[i][k] = __fmul_rn(f[k], sc);
+                a[k] = fmaxf(a[k], fabsf(v[i][k]));
+            }
         }
         *reinterpret_cast<float4*>(&part[w][4 * lane]) = make_float4(a[0], a[1], a[2], a[3]);
         __syncthreads();
@@ -519,18 +525,10 @@ __global__ void __launch_bounds__(256, 4) k_requant_128x1(const uint8_t* __restr
         uint32_t out[4][4];
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-            float v[4][4];   // [token][channel]
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int t = w * 16 + q4 * 4 + u;
-                float f[4];
-                decode4_e4m3(tw[t * (kReqCh / 4) + lane], f);
-                const float sc = sc_t[t];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) v[u][k] = __fmul_rn(f[k], sc);
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) out[k][q4] = encode4(v[0][k], v[1][k], v[2][k], v[3][k], g[k].inv);
+            for (int k = 0; k < 4; ++k)
+                out[k][q4] = encode4(v[4 * q4][k], v[4 * q4 + 1][k], v[4 * q4 + 2][k], v[4 * q4 + 3][k],
+                                     g[k].inv);
         }
         __syncthreads();   // every read of the staged codes and of part is done
         uint8_t* tl = tile[buf];
