@@ -13,8 +13,8 @@
 // accumulator living in TMEM: the MMA writes K-block kb's partial into one of
 // two TMEM buffers while the promotion warps drain the other buffer into
 // FP32 registers.  Roles per CTA (persistent, one CTA per SM):
-//   warp 0      TMA producer: A / B tiles for each K-block into a 4-stage
-//               shared-memory ring (128-byte swizzle, no cluster multicast)
+//   warp 0      TMA producer: A / B tiles for each K-block into a shared-
+//               memory ring (128-byte swizzle, no cluster multicast)
 //   warp 1      TMEM allocator + MMA issuer: 4 x tcgen05.mma (K = 32 each)
 //               per K-block into TMEM buffer kb & 1, then tcgen05.commit
 //   warps 2-3   idle (they complete warpgroup 0, which hands its registers
@@ -22,8 +22,19 @@
 //   warps 4-11  promotion + epilogue: tcgen05.ld the partial, FMA it (packed
 //               FP32x2) with its scale into a register accumulator, release the
 //               buffer; after the last K-block convert to BF16/FP32 and store.
-// Tile: 128 (M) x 256 (N) x 128 (K); warps 4-7 own columns 0-127, warps 8-11
-// columns 128-255, each warp the 32 TMEM lanes (rows) its id allows.
+// Each CTA promotes a 128 (M) x 256 (N) block; warps 4-7 own its columns
+// 0-127, warps 8-11 columns 128-255, each warp the 32 TMEM lanes (rows) its
+// id allows.
+//
+// Dense GEMMs run on CTA pairs (2-CTA clusters): one tcgen05.mma.cta_group::2
+// issued by the even CTA computes a 256 x 256 x 32 product on the tensor
+// cores of both SMs.  Each CTA loads its own 128 rows of A and 128 of B's 256
+// columns, so a K-block brings 32 KB into each SM instead of 48 KB; with the
+// bytes freed the ring holds 6 stages instead of 4.  Both CTAs' loads count
+// on the even CTA's `full` barrier, the MMA's commits arrive on both CTAs'
+// `empty` / `tfull` barriers, and every promotion warp of the pair releases a
+// TMEM buffer on the even CTA's `tempty` barrier.  Grouped (MoE) GEMMs keep
+// one CTA per 128-row block, because a 256-row pair would straddle groups.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -42,9 +53,18 @@ namespace {
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 128;
-constexpr int NS = 4;                                   // shared-memory stages
 constexpr uint32_t A_BYTES = BM * BK;                   // 16 KB per stage
-constexpr uint32_t B_BYTES = BN * BK;                   // 32 KB per stage
+constexpr uint32_t RING_BYTES = 4 * (A_BYTES + BN * BK); // 192 KB of stages
+constexpr int MAX_NS = 6;
+// Per-CTA tiling: a single CTA loads all 256 columns of B per K-block (48 KB
+// stages, 4 of them); a CTA of a pair loads 128 (32 KB stages, 6 of them).
+template <bool PAIR>
+struct Tiling {
+    static constexpr int TILE_M = PAIR ? 256 : 128;      // rows per MMA tile
+    static constexpr uint32_t B_BYTES = PAIR ? 128 * BK : BN * BK;
+    static constexpr int NS = (int)(RING_BYTES / (A_BYTES + B_BYTES));
+};
+static_assert(Tiling<true>::NS <= MAX_NS && Tiling<false>::NS <= MAX_NS, "ring barriers");
 constexpr int NUM_PROMO_WARPS = 8;
 constexpr int FIRST_PROMO_WARP = 4;                     // warpgroups 1 and 2
 constexpr int NUM_THREADS = 128 + 32 * NUM_PROMO_WARPS; // 384 = 3 warpgroups
@@ -59,7 +79,7 @@ static_assert(128 * CTRL_REGS + 256 * PROMO_REGS <= NUM_THREADS * LAUNCH_REGS,
 constexpr uint32_t TMEM_COLS = 2 * BN;                  // two FP32 partial buffers
 constexpr int MAX_GROUPS = 1024;
 constexpr int BAND = 16;                                // m-blocks per raster band
-constexpr uint32_t DYN_SMEM = 1024 + NS * (A_BYTES + B_BYTES);
+constexpr uint32_t DYN_SMEM = 1024 + RING_BYTES;
 
 struct GemmParams {
     const float* sA;               // [K/128][M]
@@ -69,7 +89,7 @@ struct GemmParams {
     int64_t M, N, K, ldd;
     int G;
     int b_major, sb_gran, out_dtype;
-    int b_box_rows;                // rows of a K-major B box (128 or 256)
+    int b_box_rows;                // rows of a K-major B box (128 or 256; 128 for pairs)
     uint64_t timeout_ns;
 };
 
@@ -77,8 +97,8 @@ struct GemmParams {
 struct __align__(16) Shared {
     float sbw[NUM_PROMO_WARPS][2][128];   // per-warp column scales (sb_gran == 1),
                                           // read and written as float4: first, 16-B aligned
-    uint64_t full[NS];
-    uint64_t empty[NS];
+    uint64_t full[MAX_NS];
+    uint64_t empty[MAX_NS];
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t drain;
@@ -99,25 +119,44 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 
 // ------------------------------------------------------------------ roles
 
+// Tiles are dealt round-robin to CTAs, or to pairs: pair c is CTAs 2c, 2c+1.
+template <bool PAIR>
+__device__ __forceinline__ void unit_range(int64_t& first, int64_t& stride)
+{
+    first = PAIR ? (int64_t)(blockIdx.x >> 1) : (int64_t)blockIdx.x;
+    stride = PAIR ? (int64_t)(gridDim.x >> 1) : (int64_t)gridDim.x;
+}
+
+template <bool PAIR>
 __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const GemmParams& p,
                              uint8_t* smem, Shared& sh, int64_t nmb, int64_t nnb, int64_t nkb)
 {
+    using T = Tiling<PAIR>;
+    constexpr int NS = T::NS;
     volatile int* abort = &sh.abort;
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
     int64_t it = 0;   // loads issued so far; stage it % NS, round it / NS
     bool ok = true;
-    for (int64_t tile = blockIdx.x; ok && tile < nmb * nnb; tile += gridDim.x) {
+    int64_t first, stride;
+    unit_range<PAIR>(first, stride);
+    for (int64_t tile = first; ok && tile < nmb * nnb; tile += stride) {
         int64_t mb, nb;
         gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
-        const int64_t m0 = mb * BM, n0 = nb * BN;
+        const int64_t m0 = mb * T::TILE_M + rank * BM;
+        const int64_t n0 = nb * BN;
         int g = 0;
-        if (p.group_offsets) {
+        if (!PAIR && p.group_offsets) {
             g = find_group(sh.off, p.G, m0);
             if (g < 0) continue;
         }
         const int64_t n_valid = (p.N - n0 < BN) ? (p.N - n0) : BN;
-        const uint32_t b_bytes = (p.b_major == FP8_B_KMAJOR) ? (uint32_t)p.b_box_rows * BK
+        // Bytes one CTA's B load(s) land per K-block (a box counts in full,
+        // its out-of-range part zero-filled).  A CTA of a pair loads B's
+        // columns rank*128 .. rank*128+127 of the tile.
+        const uint32_t b_bytes = PAIR                        ? 128u * BK
+                                 : p.b_major == FP8_B_KMAJOR ? (uint32_t)p.b_box_rows * BK
                                                              : (uint32_t)n_valid * BK;
-        const int32_t brow = (int32_t)((int64_t)g * p.N + n0);
+        const int32_t brow = (int32_t)((int64_t)g * p.N + n0 + rank * 128);
         for (int64_t kb = 0; kb < nkb; ++kb) {
             const int s = (int)(it % NS);
             const uint32_t ph = (uint32_t)((it / NS) & 1);
@@ -126,22 +165,38 @@ __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, con
                 break;
             }
             ++it;
-            mbar_arrive_expect_tx(&sh.full[s], A_BYTES + b_bytes);
             uint8_t* a_dst = smem + s * A_BYTES;
-            uint8_t* b_dst = smem + NS * A_BYTES + s * B_BYTES;
-            tma_load_2d(a_dst, tmA, &sh.full[s], (int32_t)(kb * BK), (int32_t)m0);
-            if (p.b_major == FP8_B_KMAJOR) {
-                tma_load_2d(b_dst, tmB, &sh.full[s], (int32_t)(kb * BK), brow);
+            uint8_t* b_dst = smem + NS * A_BYTES + s * T::B_BYTES;
+            if (PAIR) {
+                // Both CTAs' loads complete on the even CTA's barrier, which
+                // expects the pair's bytes; the odd CTA only issues its loads.
+                const uint32_t bar = mapa_shared(smem_u32(&sh.full[s]), 0);
+                if (rank == 0) mbar_arrive_expect_tx(&sh.full[s], 2 * (A_BYTES + b_bytes));
+                tma_load_2d_pair(a_dst, tmA, bar, (int32_t)(kb * BK), (int32_t)m0);
+                if (p.b_major == FP8_B_KMAJOR)
+                    tma_load_2d_pair(b_dst, tmB, bar, (int32_t)(kb * BK), brow);
+                else
+                    tma_load_2d_pair(b_dst, tmB, bar, (int32_t)(n0 + rank * 128),
+                                     (int32_t)(kb * BK));
             } else {
-                tma_load_2d(b_dst, tmB, &sh.full[s], (int32_t)n0, (int32_t)(kb * BK));
-                if (n_valid > 128)
-                    tma_load_2d(b_dst + 128 * BK, tmB, &sh.full[s], (int32_t)(n0 + 128),
-                                (int32_t)(kb * BK));
+                mbar_arrive_expect_tx(&sh.full[s], A_BYTES + b_bytes);
+                tma_load_2d(a_dst, tmA, &sh.full[s], (int32_t)(kb * BK), (int32_t)m0);
+                if (p.b_major == FP8_B_KMAJOR) {
+                    tma_load_2d(b_dst, tmB, &sh.full[s], (int32_t)(kb * BK), brow);
+                } else {
+                    tma_load_2d(b_dst, tmB, &sh.full[s], (int32_t)n0, (int32_t)(kb * BK));
+                    if (n_valid > 128)
+                        tma_load_2d(b_dst + 128 * BK, tmB, &sh.full[s], (int32_t)(n0 + 128),
+                                    (int32_t)(kb * BK));
+                }
             }
         }
     }
     // Every copy issued must land before the CTA may exit: stage s received
     // ceil((it - s) / NS) loads, the last one completing phase (count-1)&1.
+    // A pair's loads all count on the even CTA's barriers, so it drains for
+    // both (the odd CTA stays resident until the closing cluster barrier).
+    if (PAIR && rank != 0) return;
 #pragma unroll
     for (int s = 0; s < NS; ++s) {
         const int64_t count = it > s ? (it - s + NS - 1) / NS : 0;
@@ -149,22 +204,30 @@ __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, con
     }
 }
 
+template <bool PAIR>
 __device__ void run_mma(const GemmParams& p, uint8_t* smem, Shared& sh, int64_t nmb, int64_t nnb,
                         int64_t nkb)
 {
+    using T = Tiling<PAIR>;
+    constexpr int NS = T::NS;
     volatile int* abort = &sh.abort;
     const uint32_t a_base = smem_u32(smem);
     const uint32_t b_base = a_base + NS * A_BYTES;
     const uint32_t tmem = sh.tmem_base;
     int64_t it = 0, kbg = 0;
     bool ok = true;
-    for (int64_t tile = blockIdx.x; ok && tile < nmb * nnb; tile += gridDim.x) {
+    int64_t first, stride;
+    unit_range<PAIR>(first, stride);
+    for (int64_t tile = first; ok && tile < nmb * nnb; tile += stride) {
         int64_t mb, nb;
         gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
         const int64_t n0 = nb * BN;
-        if (p.group_offsets && find_group(sh.off, p.G, mb * BM) < 0) continue;
+        if (!PAIR && p.group_offsets && find_group(sh.off, p.G, mb * BM) < 0) continue;
         const int64_t n_valid = (p.N - n0 < BN) ? (p.N - n0) : BN;
-        const uint32_t idesc = idesc_e4m3_f32(BM, (uint32_t)n_valid, (uint32_t)p.b_major);
+        // A pair's MMA always spans 256 columns (a B tail is zero-filled).
+        const uint32_t idesc = idesc_e4m3_f32((uint32_t)T::TILE_M,
+                                              PAIR ? (uint32_t)BN : (uint32_t)n_valid,
+                                              (uint32_t)p.b_major);
         for (int64_t kb = 0; kb < nkb; ++kb, ++it, ++kbg) {
             const int s = (int)(it % NS);
             const uint32_t ph = (uint32_t)((it / NS) & 1);
@@ -178,28 +241,42 @@ __device__ void run_mma(const GemmParams& p, uint8_t* smem, Shared& sh, int64_t 
             tc_fence_after();
             const uint32_t d = tmem + buf * BN;
             const uint32_t a_addr = a_base + s * A_BYTES;
-            const uint32_t b_addr = b_base + s * B_BYTES;
+            const uint32_t b_addr = b_base + s * T::B_BYTES;
 #pragma unroll
             for (int k = 0; k < BK / 32; ++k) {
                 const uint64_t adesc = smem_desc_sw128(a_addr + k * 32, 16, 1024);
                 const uint64_t bdesc = (p.b_major == FP8_B_KMAJOR)
                                            ? smem_desc_sw128(b_addr + k * 32, 16, 1024)
                                            : smem_desc_sw128(b_addr + k * 32 * 128, 128 * BK, 1024);
-                mma_f8f6f4(d, adesc, bdesc, idesc, k > 0 ? 1u : 0u);
+                if (PAIR)
+                    mma_f8f6f4_pair(d, adesc, bdesc, idesc, k > 0 ? 1u : 0u);
+                else
+                    mma_f8f6f4(d, adesc, bdesc, idesc, k > 0 ? 1u : 0u);
             }
-            mma_commit(&sh.empty[s]);     // stage free once these MMAs are done
-            mma_commit(&sh.tfull[buf]);   // partial of this K-block ready
+            if (PAIR) {
+                // stage free and partial ready in both CTAs of the pair
+                mma_commit_pair(&sh.empty[s], 3);
+                mma_commit_pair(&sh.tfull[buf], 3);
+            } else {
+                mma_commit(&sh.empty[s]);     // stage free once these MMAs are done
+                mma_commit(&sh.tfull[buf]);   // partial of this K-block ready
+            }
         }
     }
     // Wait for every MMA this thread issued before TMEM is released.
-    mma_commit(&sh.drain);
+    if (PAIR)
+        mma_commit_pair(&sh.drain, 1);
+    else
+        mma_commit(&sh.drain);
     mbar_wait_drain(&sh.drain, 0, p.timeout_ns);
 }
 
+template <bool PAIR>
 __device__ void run_promotion(const GemmParams& p, Shared& sh, int nmb, int nnb, int nkb, int warp,
                               int lane)
 {
     volatile int* abort = &sh.abort;
+    const int rank = PAIR ? (int)cluster_ctarank() : 0;
     const int ew = warp - FIRST_PROMO_WARP;   // 0..7
     const int quad = warp & 3;            // TMEM lanes this warp may access
     const int half = ew >> 2;             // column half of the tile
@@ -209,13 +286,15 @@ __device__ void run_promotion(const GemmParams& p, Shared& sh, int nmb, int nnb,
     const int nnb128 = (int)(p.N / 128);
     uint32_t kbg = 0;
 
-    for (int tile = blockIdx.x; tile < nmb * nnb; tile += gridDim.x) {
+    int64_t first, stride;
+    unit_range<PAIR>(first, stride);
+    for (int tile = (int)first; tile < nmb * nnb; tile += (int)stride) {
         int64_t mb64, nb64;
         gemm_tile_coord(tile, nmb, nnb, BAND, mb64, nb64);
         const int mb = (int)mb64, nb = (int)nb64;
-        const int m0 = mb * BM, n0 = nb * BN;
+        const int m0 = mb * Tiling<PAIR>::TILE_M + rank * BM, n0 = nb * BN;
         int g = 0;
-        if (p.group_offsets) {
+        if (!PAIR && p.group_offsets) {
             g = find_group(sh.off, p.G, m0);
             if (g < 0) continue;
         }
@@ -315,7 +394,12 @@ __device__ void run_promotion(const GemmParams& p, Shared& sh, int nmb, int nnb,
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sh.tempty[buf]);
+            if (lane == 0) {
+                if (PAIR)   // the even CTA's MMA waits for both CTAs' warps
+                    mbar_arrive_cluster(mapa_shared(smem_u32(&sh.tempty[buf]), 0));
+                else
+                    mbar_arrive(&sh.tempty[buf]);
+            }
             if (p.sb_gran == 1) {
                 *reinterpret_cast<float4*>(&sh.sbw[ew][(kb + 1) & 1][lane * 4]) = sb4_next;
                 __syncwarp();
@@ -348,30 +432,35 @@ __device__ void run_promotion(const GemmParams& p, Shared& sh, int nmb, int nnb,
     }
 }
 
+template <bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_fp8_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const GemmParams p)
 {
+    using T = Tiling<PAIR>;
     extern __shared__ uint8_t smem_raw[];
     __shared__ Shared sh;
-    // Operand tiles need 1024-byte alignment (128-byte swizzle atoms).
+    // Operand tiles need 1024-byte alignment (128-byte swizzle atoms).  The
+    // offset is the same in both CTAs of a pair, as the pair MMA requires.
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int64_t nmb = (p.M + BM - 1) / BM;
+    const int64_t nmb = (p.M + T::TILE_M - 1) / T::TILE_M;
     const int64_t nnb = (p.N + BN - 1) / BN;
     const int64_t nkb = p.K / BK;
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < NS; ++s) {
+        for (int s = 0; s < T::NS; ++s) {
             mbar_init(&sh.full[s], 1);
             mbar_init(&sh.empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sh.tfull[b], 1);
-            mbar_init(&sh.tempty[b], NUM_PROMO_WARPS);
+            // a pair's TMEM buffer is released by the promotion warps of both CTAs
+            mbar_init(&sh.tempty[b], PAIR ? 2 * NUM_PROMO_WARPS : NUM_PROMO_WARPS);
         }
         mbar_init(&sh.drain, 1);
         sh.abort = 0;
@@ -381,17 +470,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tma_prefetch_desc(&tmB);
     }
     if (warp == 1) {
-        tmem_alloc(&sh.tmem_base, TMEM_COLS);
-        tmem_relinquish();
+        if (PAIR) {
+            tmem_alloc_pair(&sh.tmem_base, TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(&sh.tmem_base, TMEM_COLS);
+            tmem_relinquish();
+        }
     }
-    if (p.group_offsets)
+    if (!PAIR && p.group_offsets)
         for (int i = threadIdx.x; i <= p.G; i += NUM_THREADS) sh.off[i] = p.group_offsets[i];
+    // Barrier inits and the TMEM address must be visible to the peer CTA
+    // before any of its loads, commits or arrives target them.
     tc_fence_before();
-    __syncthreads();
+    if (PAIR)
+        cluster_sync();
+    else
+        __syncthreads();
     tc_fence_after();
-    if (p.group_offsets && threadIdx.x == 0) {
+    if (!PAIR && p.group_offsets && threadIdx.x == 0) {
         bool bad = sh.off[0] != 0 || (int64_t)sh.off[p.G] > p.M;
-        for (int e = 0; e < p.G; ++e) bad = bad || sh.off[e + 1] < sh.off[e] || (sh.off[e + 1] & 127);
+        for (int e = 0; e < p.G; ++e)
+            bad = bad || sh.off[e + 1] < sh.off[e] || (sh.off[e + 1] & 127);
         if (bad) {
             sh.bad = 1;
             if (blockIdx.x == 0) report_error(FP8_ERR_SHAPE);
@@ -403,21 +503,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         regs_dec<CTRL_REGS>();
         if (!sh.bad) {
             if (warp == 0) {
-                if (lane == 0) run_producer(&tmA, &tmB, p, smem, sh, nmb, nnb, nkb);
+                if (lane == 0) run_producer<PAIR>(&tmA, &tmB, p, smem, sh, nmb, nnb, nkb);
                 __syncwarp();
-            } else if (warp == 1) {
-                if (lane == 0) run_mma(p, smem, sh, nmb, nnb, nkb);
+            } else if (warp == 1 && rank == 0) {   // a pair's MMAs issue from the even CTA
+                if (lane == 0) run_mma<PAIR>(p, smem, sh, nmb, nnb, nkb);
                 __syncwarp();
             }
         }
     } else {
         regs_inc<PROMO_REGS>();
-        if (!sh.bad) run_promotion(p, sh, (int)nmb, (int)nnb, (int)nkb, warp, lane);
+        if (!sh.bad) run_promotion<PAIR>(p, sh, (int)nmb, (int)nnb, (int)nkb, warp, lane);
     }
     tc_fence_before();
-    __syncthreads();
+    if (PAIR)
+        cluster_sync();
+    else
+        __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(sh.tmem_base, TMEM_COLS);
+    if (warp == 1) {
+        if (PAIR)
+            tmem_dealloc_pair(sh.tmem_base, TMEM_COLS);
+        else
+            tmem_dealloc(sh.tmem_base, TMEM_COLS);
+    }
 }
 
 __global__ void k_selftest_wait(uint64_t timeout_ns)
@@ -436,21 +544,59 @@ __global__ void k_selftest_wait(uint64_t timeout_ns)
 
 // ------------------------------------------------------------------ host side
 
-bool ensure_smem_attr()
+cudaLaunchConfig_t pair_launch_config(unsigned clusters, cudaStream_t st, cudaLaunchAttribute* attr)
 {
-    // once per device
-    static bool done[64] = {};
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * clusters, 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = DYN_SMEM;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cfg;
+}
+
+// Once per device: opt both kernels into the large dynamic shared memory and
+// ask how many CTA pairs fit at once (the persistent grid of the pair kernel;
+// 0 means pairs are unavailable and dense GEMMs run on single CTAs).
+struct GemmDeviceSetup {
+    bool ok = false;
+    int pair_clusters = 0;
+};
+
+GemmDeviceSetup gemm_device_setup()
+{
+    static GemmDeviceSetup done[64];
+    static bool tried[64] = {};
     static std::mutex mu;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GemmDeviceSetup{};
     std::lock_guard<std::mutex> lk(mu);
-    if (!done[dev]) {
-        if (cudaFuncSetAttribute(k_fp8_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)DYN_SMEM) != cudaSuccess)
-            return false;
-        done[dev] = true;
+    if (!tried[dev]) {
+        tried[dev] = true;
+        GemmDeviceSetup r;
+        r.ok = cudaFuncSetAttribute(k_fp8_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)DYN_SMEM) == cudaSuccess &&
+               cudaFuncSetAttribute(k_fp8_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)DYN_SMEM) == cudaSuccess;
+        if (r.ok) {
+            cudaLaunchAttribute attr[1];
+            const cudaLaunchConfig_t cfg =
+                pair_launch_config((unsigned)device_sm_count(), nullptr, attr);
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, k_fp8_gemm<true>, &cfg) != cudaSuccess) {
+                n = 0;
+                (void)cudaGetLastError();
+            }
+            r.pair_clusters = n;
+        }
+        done[dev] = r;
     }
-    return true;
+    return done[dev];
 }
 
 }  // namespace
@@ -497,8 +643,12 @@ int launch_blockscaled_gemm(const uint8_t* A, const float* sA, const uint8_t* B,
                             int64_t ldd, cudaStream_t st)
 {
     if (M == 0) return FP8_OK;
+    const GemmDeviceSetup setup = gemm_device_setup();
+    if (!setup.ok) return FP8_ERR_LAUNCH;
+    // Dense GEMMs run on CTA pairs; grouped ones keep 128-row single CTAs.
+    const bool pair = group_offsets == nullptr && setup.pair_clusters > 0;
     CUtensorMap tmA, tmB;
-    const int b_box_rows = N >= BN ? BN : (int)N;
+    const int b_box_rows = pair ? 128 : (N >= BN ? BN : (int)N);
     if (!make_map(&tmA, A, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, BM)) return FP8_ERR_LAUNCH;
     bool okB;
     if (b_major == FP8_B_KMAJOR) {
@@ -508,8 +658,6 @@ int launch_blockscaled_gemm(const uint8_t* A, const float* sA, const uint8_t* B,
         okB = make_map(&tmB, B, (uint64_t)N, (uint64_t)K, (uint64_t)N, 128, BK);
     }
     if (!okB) return FP8_ERR_LAUNCH;
-    if (!ensure_smem_attr()) return FP8_ERR_LAUNCH;
-
     GemmParams p;
     p.sA = sA;
     p.sB = sB;
@@ -525,11 +673,19 @@ int launch_blockscaled_gemm(const uint8_t* A, const float* sA, const uint8_t* B,
     p.out_dtype = out_dtype;
     p.b_box_rows = b_box_rows;
     p.timeout_ns = wait_timeout_ns();
-
+    if (pair) {
+        const int64_t tiles = ((M + 255) / 256) * ((N + BN - 1) / BN);
+        const int64_t clusters = tiles < setup.pair_clusters ? tiles : setup.pair_clusters;
+        cudaLaunchAttribute attr[1];
+        const cudaLaunchConfig_t cfg = pair_launch_config((unsigned)clusters, st, attr);
+        return cudaLaunchKernelEx(&cfg, k_fp8_gemm<true>, tmA, tmB, p) == cudaSuccess
+                   ? FP8_OK
+                   : FP8_ERR_LAUNCH;
+    }
     const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
     const int sms = device_sm_count();
     const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
-    k_fp8_gemm<<<grid, NUM_THREADS, DYN_SMEM, st>>>(tmA, tmB, p);
+    k_fp8_gemm<false><<<grid, NUM_THREADS, DYN_SMEM, st>>>(tmA, tmB, p);
     return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_LAUNCH;
 }
 
