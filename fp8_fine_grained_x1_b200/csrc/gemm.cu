@@ -364,7 +364,7 @@ __device__ void run_promotion(const GemmParams& p, Shared& sh, int nmb, int nnb,
                     for (int c = 0; c < 8; ++c) {
                         uint32_t r[16];
                         tmem_ld16(taddr + c * 16, r);
-                        tmem_ld_wait();
+                        tmem_ld_wait(r);
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
                             ffma2(acc[c * 16 + 2 * i], acc[c * 16 + 2 * i + 1],
@@ -376,7 +376,7 @@ __device__ void run_promotion(const GemmParams& p, Shared& sh, int nmb, int nnb,
                     for (int c = 0; c < 8; ++c) {
                         uint32_t r[16];
                         tmem_ld16(taddr + c * 16, r);
-                        tmem_ld_wait();
+                        tmem_ld_wait(r);
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             const float4 b = *reinterpret_cast<const float4*>(sbv + c * 16 + 4 * i);

@@ -414,7 +414,7 @@ __device__ void mx_epilogue(const MxParams& p, MxShared& sh, int64_t nmb, int64_
             uint32_t r[32];
             if (active) {
                 tmem_ld32(taddr0 + (uint32_t)(c * 32), r);
-                tmem_ld_wait();
+                tmem_ld_wait(r);
             }
             if (c == 3) {                        // accumulator no longer needed
                 tc_fence_before();

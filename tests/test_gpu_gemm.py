@@ -52,6 +52,11 @@ CASES = [
     (200, 384, 512, fg.B_MNMAJOR, 128),
     (128, 256, 512, fg.B_KMAJOR, 1),          # Wgrad layout (per-column B scales)
     (256, 384, 1024, fg.B_KMAJOR, 1),
+    # 256-row tiles of CTA pairs: the odd CTA's 128 rows wholly beyond M, and
+    # a last n-tile whose second 128 columns lie beyond N
+    (384, 640, 384, fg.B_KMAJOR, 1),
+    (384, 640, 256, fg.B_MNMAJOR, 128),
+    (300, 640, 256, fg.B_KMAJOR, 128),
 ]
 
 
