@@ -33,8 +33,11 @@
 // bytes freed the ring holds 6 stages instead of 4.  Both CTAs' loads count
 // on the even CTA's `full` barrier, the MMA's commits arrive on both CTAs'
 // `empty` / `tfull` barriers, and every promotion warp of the pair releases a
-// TMEM buffer on the even CTA's `tempty` barrier.  Grouped (MoE) GEMMs keep
-// one CTA per 128-row block, because a 256-row pair would straddle groups.
+// TMEM buffer on the even CTA's `tempty` barrier.  Grouped (MoE) GEMMs count
+// their 256-row blocks group by group, so that both halves of a pair use the
+// same expert's B; a group of an odd number of 128-row blocks leaves the odd
+// CTA of its last pair idle.  Single CTAs remain the fallback when the device
+// cannot co-schedule 2-CTA clusters.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -76,6 +79,7 @@ constexpr uint32_t CTRL_REGS = 40;
 constexpr uint32_t PROMO_REGS = 216;
 static_assert(128 * CTRL_REGS + 256 * PROMO_REGS <= NUM_THREADS * LAUNCH_REGS,
               "register split exceeds the launch allocation");
+constexpr int PROMO_CHUNK = 32;                        // TMEM columns per load round trip
 constexpr uint32_t TMEM_COLS = 2 * BN;                  // two FP32 partial buffers
 constexpr int MAX_GROUPS = 1024;
 constexpr int BAND = 16;                                // m-blocks per raster band
@@ -105,7 +109,8 @@ struct __align__(16) Shared {
     uint32_t tmem_base;
     int abort;
     int bad;
-    int32_t off[MAX_GROUPS + 1];
+    int32_t off[MAX_GROUPS + 1];    // grouped: row offsets of the groups
+    int32_t poff[MAX_GROUPS + 1];   // grouped pairs: first 256-row block of each group
 };
 static_assert(offsetof(Shared, sbw) % 16 == 0, "float4 accesses need 16-byte alignment");
 static_assert(sizeof(float) * 128 % 16 == 0, "per-warp scale rows stay 16-byte aligned");
@@ -118,6 +123,38 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 }
 
 // ------------------------------------------------------------------ roles
+
+// The 128 rows of A (and of D) one CTA works on in m-block mb.
+//   dense            m0 = mb * TILE_M + rank * 128, rows below M valid.
+//   grouped, single  m0 = mb * 128, in the group holding that row; blocks at
+//                    or past off[G] hold no group and are skipped.
+//   grouped, pairs   mb counts 256-row blocks group by group (poff), so a
+//                    pair never mixes two groups' rows (it shares one B); in
+//                    a group whose row count is an odd multiple of 128 the
+//                    last pair's odd CTA lies past the group end and idles.
+struct TileRows {
+    int g;           // group (0 when dense)
+    int64_t m0;      // first row of this CTA's 128
+    int64_t m_end;   // rows m0 .. m_end-1 belong to the tile's group
+};
+
+template <bool PAIR>
+__device__ __forceinline__ bool tile_rows(const GemmParams& p, const Shared& sh, int64_t mb,
+                                          uint32_t rank, TileRows& t)
+{
+    if (!p.group_offsets) {
+        t.g = 0;
+        t.m0 = mb * Tiling<PAIR>::TILE_M + rank * BM;
+        t.m_end = p.M;
+        return true;
+    }
+    const int g = PAIR ? find_group(sh.poff, p.G, mb) : find_group(sh.off, p.G, mb * BM);
+    if (g < 0) return false;
+    t.g = g;
+    t.m0 = PAIR ? sh.off[g] + (mb - sh.poff[g]) * 256 + rank * BM : mb * BM;
+    t.m_end = sh.off[g + 1];
+    return true;
+}
 
 // Tiles are dealt round-robin to CTAs, or to pairs: pair c is CTAs 2c, 2c+1.
 template <bool PAIR>
@@ -142,13 +179,12 @@ __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, con
     for (int64_t tile = first; ok && tile < nmb * nnb; tile += stride) {
         int64_t mb, nb;
         gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
-        const int64_t m0 = mb * T::TILE_M + rank * BM;
+        TileRows tr;
+        if (!tile_rows<PAIR>(p, sh, mb, rank, tr)) continue;
+        // (an idle odd CTA still loads its rows: the pair's MMA counts them)
+        const int64_t m0 = tr.m0;
         const int64_t n0 = nb * BN;
-        int g = 0;
-        if (!PAIR && p.group_offsets) {
-            g = find_group(sh.off, p.G, m0);
-            if (g < 0) continue;
-        }
+        const int g = tr.g;
         const int64_t n_valid = (p.N - n0 < BN) ? (p.N - n0) : BN;
         // Bytes one CTA's B load(s) land per K-block (a box counts in full,
         // its out-of-range part zero-filled).  A CTA of a pair loads B's
@@ -291,16 +327,16 @@ __device__ void run_promotion(const GemmParams& p, Shared& sh, int nmb, int nnb,
     for (int tile = (int)first; tile < nmb * nnb; tile += (int)stride) {
         int64_t mb64, nb64;
         gemm_tile_coord(tile, nmb, nnb, BAND, mb64, nb64);
-        const int mb = (int)mb64, nb = (int)nb64;
-        const int m0 = mb * Tiling<PAIR>::TILE_M + rank * BM, n0 = nb * BN;
-        int g = 0;
-        if (!PAIR && p.group_offsets) {
-            g = find_group(sh.off, p.G, m0);
-            if (g < 0) continue;
-        }
+        TileRows tr;
+        if (!tile_rows<PAIR>(p, sh, mb64, (uint32_t)rank, tr)) continue;
+        const int nb = (int)nb64;
+        const int m0 = (int)tr.m0, n0 = nb * BN;
+        const int g = tr.g;
         const int m = m0 + row;
-        const bool row_ok = m < p.M;
-        const bool active = (n0 + col0) < p.N;
+        const bool row_ok = m < tr.m_end;
+        // a warp whose columns lie past N, or whose CTA idles in this tile,
+        // only keeps the K-block handshakes going
+        const bool active = (n0 + col0) < p.N && tr.m0 < tr.m_end;
         const int cb = (n0 + col0) / 128;   // 128-column block of B
 
         // Scales of K-block kb for this thread, prefetched one K-block ahead:
@@ -358,37 +394,50 @@ __device__ void run_promotion(const GemmParams& p, Shared& sh, int nmb, int nnb,
             tc_fence_after();
             if (active) {
                 const uint32_t taddr = tmem_lane + buf * BN + col0;
+                // PROMO_CHUNK columns per TMEM round trip: their 16-column
+                // loads are all in flight before the first wait.
+                constexpr int NL = PROMO_CHUNK / 16;
                 if (p.sb_gran == 128) {
                     const float sc = sa * sb;
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        uint32_t r[16];
-                        tmem_ld16(taddr + c * 16, r);
-                        tmem_ld_wait(r);
+                    for (int c = 0; c < 128 / PROMO_CHUNK; ++c) {
+                        uint32_t r[NL][16];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            ffma2(acc[c * 16 + 2 * i], acc[c * 16 + 2 * i + 1],
-                                  __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), sc, sc);
+                        for (int l = 0; l < NL; ++l) tmem_ld16(taddr + c * PROMO_CHUNK + l * 16, r[l]);
+#pragma unroll
+                        for (int l = 0; l < NL; ++l) tmem_ld_wait(r[l]);
+#pragma unroll
+                        for (int l = 0; l < NL; ++l)
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const int j = c * PROMO_CHUNK + l * 16 + 2 * i;
+                                ffma2(acc[j], acc[j + 1], __uint_as_float(r[l][2 * i]),
+                                      __uint_as_float(r[l][2 * i + 1]), sc, sc);
+                            }
                     }
                 } else {
                     const float* sbv = sh.sbw[ew][kb & 1];
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        uint32_t r[16];
-                        tmem_ld16(taddr + c * 16, r);
-                        tmem_ld_wait(r);
+                    for (int c = 0; c < 128 / PROMO_CHUNK; ++c) {
+                        uint32_t r[NL][16];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float4 b = *reinterpret_cast<const float4*>(sbv + c * 16 + 4 * i);
-                            float t0, t1, t2, t3;
-                            fmul2(t0, t1, b.x, b.y, sa, sa);
-                            fmul2(t2, t3, b.z, b.w, sa, sa);
-                            const int j = c * 16 + 4 * i;
-                            ffma2(acc[j], acc[j + 1], __uint_as_float(r[4 * i]),
-                                  __uint_as_float(r[4 * i + 1]), t0, t1);
-                            ffma2(acc[j + 2], acc[j + 3], __uint_as_float(r[4 * i + 2]),
-                                  __uint_as_float(r[4 * i + 3]), t2, t3);
-                        }
+                        for (int l = 0; l < NL; ++l) tmem_ld16(taddr + c * PROMO_CHUNK + l * 16, r[l]);
+#pragma unroll
+                        for (int l = 0; l < NL; ++l) tmem_ld_wait(r[l]);
+#pragma unroll
+                        for (int l = 0; l < NL; ++l)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int j = c * PROMO_CHUNK + l * 16 + 4 * i;
+                                const float4 b = *reinterpret_cast<const float4*>(sbv + j);
+                                float t0, t1, t2, t3;
+                                fmul2(t0, t1, b.x, b.y, sa, sa);
+                                fmul2(t2, t3, b.z, b.w, sa, sa);
+                                ffma2(acc[j], acc[j + 1], __uint_as_float(r[l][4 * i]),
+                                      __uint_as_float(r[l][4 * i + 1]), t0, t1);
+                                ffma2(acc[j + 2], acc[j + 3], __uint_as_float(r[l][4 * i + 2]),
+                                      __uint_as_float(r[l][4 * i + 3]), t2, t3);
+                            }
                     }
                 }
             }
@@ -447,7 +496,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int64_t nmb = (p.M + T::TILE_M - 1) / T::TILE_M;
     const int64_t nnb = (p.N + BN - 1) / BN;
     const int64_t nkb = p.K / BK;
     const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
@@ -478,7 +526,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tmem_relinquish();
         }
     }
-    if (!PAIR && p.group_offsets)
+    if (p.group_offsets)
         for (int i = threadIdx.x; i <= p.G; i += NUM_THREADS) sh.off[i] = p.group_offsets[i];
     // Barrier inits and the TMEM address must be visible to the peer CTA
     // before any of its loads, commits or arrives target them.
@@ -488,7 +536,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     else
         __syncthreads();
     tc_fence_after();
-    if (!PAIR && p.group_offsets && threadIdx.x == 0) {
+    if (p.group_offsets && threadIdx.x == 0) {
         bool bad = sh.off[0] != 0 || (int64_t)sh.off[p.G] > p.M;
         for (int e = 0; e < p.G; ++e)
             bad = bad || sh.off[e + 1] < sh.off[e] || (sh.off[e + 1] & 127);
@@ -498,6 +546,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     }
     __syncthreads();
+    if (PAIR && p.group_offsets && !sh.bad && warp == 0) {
+        // poff[e] = 256-row blocks of groups 0 .. e-1: each lane sums a run of
+        // groups, a warp scan turns the sums into the runs' starting blocks.
+        const int per = (p.G + 31) / 32;
+        const int e0 = lane * per < p.G ? lane * per : p.G;
+        const int e1 = e0 + per < p.G ? e0 + per : p.G;
+        int sum = 0;
+        for (int e = e0; e < e1; ++e) sum += (sh.off[e + 1] - sh.off[e] + 255) >> 8;
+        int incl = sum;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += t;
+        }
+        int run = incl - sum;
+        for (int e = e0; e < e1; ++e) {
+            sh.poff[e] = run;
+            run += (sh.off[e + 1] - sh.off[e] + 255) >> 8;
+        }
+        if (lane == 31) sh.poff[p.G] = incl;
+    }
+    __syncthreads();
+    const int64_t nmb = (PAIR && p.group_offsets) ? (int64_t)sh.poff[p.G]
+                                                  : (p.M + T::TILE_M - 1) / T::TILE_M;
 
     if (warp < FIRST_PROMO_WARP) {
         regs_dec<CTRL_REGS>();
@@ -645,8 +717,7 @@ int launch_blockscaled_gemm(const uint8_t* A, const float* sA, const uint8_t* B,
     if (M == 0) return FP8_OK;
     const GemmDeviceSetup setup = gemm_device_setup();
     if (!setup.ok) return FP8_ERR_LAUNCH;
-    // Dense GEMMs run on CTA pairs; grouped ones keep 128-row single CTAs.
-    const bool pair = group_offsets == nullptr && setup.pair_clusters > 0;
+    const bool pair = setup.pair_clusters > 0;
     CUtensorMap tmA, tmB;
     const int b_box_rows = pair ? 128 : (N >= BN ? BN : (int)N);
     if (!make_map(&tmA, A, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, BM)) return FP8_ERR_LAUNCH;
@@ -674,7 +745,8 @@ int launch_blockscaled_gemm(const uint8_t* A, const float* sA, const uint8_t* B,
     p.b_box_rows = b_box_rows;
     p.timeout_ns = wait_timeout_ns();
     if (pair) {
-        const int64_t tiles = ((M + 255) / 256) * ((N + BN - 1) / BN);
+        // grouped: each group adds at most one partly idle 256-row block
+        const int64_t tiles = ((M + 255) / 256 + (group_offsets ? G : 0)) * ((N + BN - 1) / BN);
         const int64_t clusters = tiles < setup.pair_clusters ? tiles : setup.pair_clusters;
         cudaLaunchAttribute attr[1];
         const cudaLaunchConfig_t cfg = pair_launch_config((unsigned)clusters, st, attr);
