@@ -454,6 +454,63 @@ __device__ __forceinline__ int find_group(const int32_t* off, int G, int64_t row
     return lo < G ? lo : -1;
 }
 
+// The 128 rows of A (and of D) one CTA works on in m-block mb.
+//   dense            m0 = mb * tile_m + rank * 128, rows below M valid.
+//   grouped, single  m0 = mb * 128, in the group holding that row; blocks at
+//                    or past off[G] hold no group and are skipped (false).
+//   grouped, pairs   mb counts 256-row blocks group by group (poff), so a
+//                    pair never mixes two groups' rows (it shares one B); in
+//                    a group whose row count is an odd multiple of 128 the
+//                    last pair's odd CTA lies past the group end and idles.
+struct TileRows {
+    int g;           // group (0 when dense)
+    int64_t m0;      // first row of this CTA's 128
+    int64_t m_end;   // rows m0 .. m_end-1 belong to the tile's group
+};
+
+template <bool PAIR>
+__device__ __forceinline__ bool tile_rows(const int32_t* group_offsets, const int32_t* off,
+                                          const int32_t* poff, int G, int64_t M, int64_t mb,
+                                          uint32_t rank, TileRows& t)
+{
+    if (!group_offsets) {
+        t.g = 0;
+        t.m0 = mb * (PAIR ? 256 : 128) + rank * 128;
+        t.m_end = M;
+        return true;
+    }
+    const int g = PAIR ? find_group(poff, G, mb) : find_group(off, G, mb * 128);
+    if (g < 0) return false;
+    t.g = g;
+    t.m0 = PAIR ? off[g] + (mb - poff[g]) * 256 + rank * 128 : mb * 128;
+    t.m_end = off[g + 1];
+    return true;
+}
+
+// One warp: poff[e] = number of 256-row blocks in groups 0 .. e-1 (row
+// counts off[e+1] - off[e]), poff[G] their total.  Each lane sums a run of
+// groups; a warp scan turns the sums into the runs' first blocks.
+__device__ __forceinline__ void pair_block_offsets(const int32_t* off, int32_t* poff, int G, int lane)
+{
+    const int per = (G + 31) / 32;
+    const int e0 = lane * per < G ? lane * per : G;
+    const int e1 = e0 + per < G ? e0 + per : G;
+    int sum = 0;
+    for (int e = e0; e < e1; ++e) sum += (off[e + 1] - off[e] + 255) >> 8;
+    int incl = sum;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += t;
+    }
+    int run = incl - sum;
+    for (int e = e0; e < e1; ++e) {
+        poff[e] = run;
+        run += (off[e + 1] - off[e] + 255) >> 8;
+    }
+    if (lane == 31) poff[G] = incl;
+}
+
 // Host: 2-D uint8 tensor map [outer][inner], rows `row_bytes` apart, boxes of
 // box_inner x box_outer bytes, 128-byte swizzle, zero fill out of bounds
 // (defined in gemm.cu; false when the driver's encoder is unavailable).

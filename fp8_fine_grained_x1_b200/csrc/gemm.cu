@@ -124,36 +124,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 
 // ------------------------------------------------------------------ roles
 
-// The 128 rows of A (and of D) one CTA works on in m-block mb.
-//   dense            m0 = mb * TILE_M + rank * 128, rows below M valid.
-//   grouped, single  m0 = mb * 128, in the group holding that row; blocks at
-//                    or past off[G] hold no group and are skipped.
-//   grouped, pairs   mb counts 256-row blocks group by group (poff), so a
-//                    pair never mixes two groups' rows (it shares one B); in
-//                    a group whose row count is an odd multiple of 128 the
-//                    last pair's odd CTA lies past the group end and idles.
-struct TileRows {
-    int g;           // group (0 when dense)
-    int64_t m0;      // first row of this CTA's 128
-    int64_t m_end;   // rows m0 .. m_end-1 belong to the tile's group
-};
-
 template <bool PAIR>
 __device__ __forceinline__ bool tile_rows(const GemmParams& p, const Shared& sh, int64_t mb,
                                           uint32_t rank, TileRows& t)
 {
-    if (!p.group_offsets) {
-        t.g = 0;
-        t.m0 = mb * Tiling<PAIR>::TILE_M + rank * BM;
-        t.m_end = p.M;
-        return true;
-    }
-    const int g = PAIR ? find_group(sh.poff, p.G, mb) : find_group(sh.off, p.G, mb * BM);
-    if (g < 0) return false;
-    t.g = g;
-    t.m0 = PAIR ? sh.off[g] + (mb - sh.poff[g]) * 256 + rank * BM : mb * BM;
-    t.m_end = sh.off[g + 1];
-    return true;
+    return tile_rows<PAIR>(p.group_offsets, sh.off, sh.poff, p.G, p.M, mb, rank, t);
 }
 
 // Tiles are dealt round-robin to CTAs, or to pairs: pair c is CTAs 2c, 2c+1.
@@ -546,27 +521,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     }
     __syncthreads();
-    if (PAIR && p.group_offsets && !sh.bad && warp == 0) {
-        // poff[e] = 256-row blocks of groups 0 .. e-1: each lane sums a run of
-        // groups, a warp scan turns the sums into the runs' starting blocks.
-        const int per = (p.G + 31) / 32;
-        const int e0 = lane * per < p.G ? lane * per : p.G;
-        const int e1 = e0 + per < p.G ? e0 + per : p.G;
-        int sum = 0;
-        for (int e = e0; e < e1; ++e) sum += (sh.off[e + 1] - sh.off[e] + 255) >> 8;
-        int incl = sum;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const int t = __shfl_up_sync(0xffffffffu, incl, d);
-            if (lane >= d) incl += t;
-        }
-        int run = incl - sum;
-        for (int e = e0; e < e1; ++e) {
-            sh.poff[e] = run;
-            run += (sh.off[e + 1] - sh.off[e] + 255) >> 8;
-        }
-        if (lane == 31) sh.poff[p.G] = incl;
-    }
+    if (PAIR && p.group_offsets && !sh.bad && warp == 0)
+        pair_block_offsets(sh.off, sh.poff, p.G, lane);
     __syncthreads();
     const int64_t nmb = (PAIR && p.group_offsets) ? (int64_t)sh.poff[p.G]
                                                   : (p.M + T::TILE_M - 1) / T::TILE_M;

@@ -15,8 +15,8 @@
 // tensor core until the tile's last K-block: there is no promotion step.
 //
 // Roles per CTA (persistent, one CTA per SM, 512 threads):
-//   warp 0      TMA producer: A / B tiles per K-block into a 4-stage ring
-//               (128-byte swizzle, no cluster multicast)
+//   warp 0      TMA producer: A / B tiles per K-block into a shared-memory
+//               ring (128-byte swizzle, no cluster multicast)
 //   warp 1      MMA issuer: 4 x block-scaled MMA (K = 32) per K-block into
 //               one TMEM accumulator, tcgen05.commit frees the stage
 //   warp 2      TMEM allocator
@@ -40,6 +40,16 @@
 // four columns wide -- exactly the layout above.  (Writing TMEM with
 // tcgen05.st from the scale warps instead measured 24 % tensor-pipe
 // activity: the stores and the MMAs contend for TMEM.)
+//
+// CTA pairs (2-CTA clusters), as in gemm.cu: the even CTA issues one
+// tcgen05.mma.cta_group::2 of 256 x 256 x 32 over both SMs; each CTA loads
+// its own 128 rows of A and 128 of B's columns.  Each SM multiplies its own
+// 128 rows by all 256 columns, so each CTA's TMEM holds the scale factors
+// of its own rows (SFA) and of all 256 columns (SFB): the scale writers of
+// both CTAs fill their own shared memory, and the even CTA's
+// tcgen05.cp.cta_group::2 moves each CTA's block into that CTA's TMEM.
+// Both CTAs' loads and scale writers count on the even CTA's `full`
+// barrier; its commits arrive on both CTAs' `empty` and `acc_full`.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -57,9 +67,7 @@ namespace {
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 128;
-constexpr int NS = 4;
 constexpr uint32_t A_BYTES = BM * BK;
-constexpr uint32_t B_BYTES = BN * BK;
 constexpr int NUM_THREADS = 512;
 constexpr int FIRST_SF_WARP = 4;
 constexpr int FIRST_EPI_WARP = 8;
@@ -69,13 +77,24 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_COL0 = BN;
 constexpr uint32_t SF_SLOT_COLS = 16;
 constexpr uint32_t SFB_OFF = 8;
-static_assert(SF_COL0 + NS * SF_SLOT_COLS <= TMEM_COLS, "scale slots exceed the allocation");
 constexpr int BAND = 16;
 constexpr int SF_AHEAD = 4;                 // K-blocks of scales each writer loads ahead
 constexpr uint32_t SFA_BYTES = 512;              // 128 rows x 4 bytes
 constexpr uint32_t SFB_BYTES = 1024;             // 256 columns x 4 bytes
 constexpr uint32_t SF_BYTES = SFA_BYTES + SFB_BYTES;
-constexpr uint32_t DYN_SMEM = 1024 + NS * (A_BYTES + B_BYTES + SF_BYTES);
+constexpr int MAX_NS = 6;
+constexpr uint32_t RING_BYTES = MAX_NS * (A_BYTES + 128 * BK + SF_BYTES);   // 201 KB
+// Per-CTA tiling: a single CTA loads all 256 columns of B per K-block (4
+// stages); a CTA of a pair loads 128 (6 stages).
+template <bool PAIR>
+struct MxTiling {
+    static constexpr int TILE_M = PAIR ? 256 : 128;
+    static constexpr uint32_t B_BYTES = PAIR ? 128 * BK : BN * BK;
+    static constexpr int NS = (int)(RING_BYTES / (A_BYTES + B_BYTES + SF_BYTES));
+};
+static_assert(MxTiling<true>::NS <= MAX_NS && MxTiling<false>::NS <= MAX_NS, "ring barriers");
+static_assert(SF_COL0 + MAX_NS * SF_SLOT_COLS <= TMEM_COLS, "scale slots exceed the allocation");
+constexpr uint32_t DYN_SMEM = 1024 + RING_BYTES;
 
 constexpr int MAX_GROUPS = 1024;
 
@@ -92,8 +111,8 @@ struct MxParams {
 };
 
 struct __align__(8) MxShared {
-    uint64_t full[NS];     // operands landed (TMA bytes) and scales stored (4 scale warps)
-    uint64_t empty[NS];
+    uint64_t full[MAX_NS];     // operands landed (TMA bytes) and scales stored (scale warps)
+    uint64_t empty[MAX_NS];
     uint64_t acc_full;
     uint64_t acc_empty;
     uint64_t drain;
@@ -101,6 +120,7 @@ struct __align__(8) MxShared {
     int abort;
     int bad;
     int32_t off[MAX_GROUPS + 1];   // grouped: the group offsets, validated on the device
+    int32_t poff[MAX_GROUPS + 1];  // grouped pairs: first 256-row block of each group
 };
 
 // -------------------------------------------------------------- PTX helpers
@@ -115,6 +135,21 @@ __device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t a_desc, uint6
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::
+            "r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// The same over a CTA pair (M = 256: rows 0-127 in the even CTA, issued by
+// it; each CTA's scale factors from its own TMEM).
+__device__ __forceinline__ void mma_mxf8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                              uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::
             "r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
         : "memory");
@@ -143,6 +178,16 @@ __device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint32_t sadd
     const uint64_t desc = (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)(16 >> 4) << 16) |
                           ((uint64_t)(128 >> 4) << 32) | ((uint64_t)1 << 46);
     asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc)
+                 : "memory");
+}
+
+// The same for a CTA pair, issued by the even CTA: each CTA's 512-byte
+// block at `saddr` goes to that CTA's TMEM at `taddr`.
+__device__ __forceinline__ void tmem_cp_32x128b_x4_pair(uint32_t taddr, uint32_t saddr)
+{
+    const uint64_t desc = (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)(16 >> 4) << 16) |
+                          ((uint64_t)(128 >> 4) << 32) | ((uint64_t)1 << 46);
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc)
                  : "memory");
 }
 
@@ -183,25 +228,44 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 
 // ------------------------------------------------------------------ roles
 
+template <bool PAIR>
+__device__ __forceinline__ bool mx_tile_rows(const MxParams& p, const MxShared& sh, int64_t mb,
+                                             uint32_t rank, TileRows& t)
+{
+    return tile_rows<PAIR>(p.group_offsets, sh.off, sh.poff, p.G, p.M, mb, rank, t);
+}
+
+// Tiles are dealt round-robin to CTAs, or to pairs: pair c is CTAs 2c, 2c+1.
+template <bool PAIR>
+__device__ __forceinline__ void mx_unit_range(int64_t& first, int64_t& stride)
+{
+    first = PAIR ? (int64_t)(blockIdx.x >> 1) : (int64_t)blockIdx.x;
+    stride = PAIR ? (int64_t)(gridDim.x >> 1) : (int64_t)gridDim.x;
+}
+
+template <bool PAIR>
 __device__ void mx_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const MxParams& p,
                             uint8_t* smem, MxShared& sh, int64_t nmb, int64_t nnb, int64_t nkb)
 {
+    using T = MxTiling<PAIR>;
+    constexpr int NS = T::NS;
     volatile int* abort = &sh.abort;
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
     int64_t it = 0;
     bool ok = true;
-    for (int64_t tile = blockIdx.x; ok && tile < nmb * nnb; tile += gridDim.x) {
+    int64_t first, stride;
+    mx_unit_range<PAIR>(first, stride);
+    for (int64_t tile = first; ok && tile < nmb * nnb; tile += stride) {
         int64_t mb, nb;
         gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
-        const int64_t m0 = mb * BM, n0 = nb * BN;
-        int g = 0;
-        if (p.group_offsets) {
-            g = find_group(sh.off, p.G, m0);
-            if (g < 0) continue;
-        }
+        TileRows tr;
+        if (!mx_tile_rows<PAIR>(p, sh, mb, rank, tr)) continue;
+        const int64_t m0 = tr.m0, n0 = nb * BN;   // an idle odd CTA still loads
         const int64_t n_valid = (p.N - n0 < BN) ? (p.N - n0) : BN;
-        const uint32_t b_bytes = (p.b_major == FP8_B_KMAJOR) ? (uint32_t)p.b_box_rows * BK
+        const uint32_t b_bytes = PAIR                        ? 128u * BK
+                                 : p.b_major == FP8_B_KMAJOR ? (uint32_t)p.b_box_rows * BK
                                                              : (uint32_t)n_valid * BK;
-        const int32_t brow = (int32_t)((int64_t)g * p.N + n0);
+        const int32_t brow = (int32_t)((int64_t)tr.g * p.N + n0 + rank * 128);
         for (int64_t kb = 0; kb < nkb; ++kb) {
             const int s = (int)(it % NS);
             const uint32_t ph = (uint32_t)((it / NS) & 1);
@@ -210,21 +274,35 @@ __device__ void mx_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, cons
                 break;
             }
             ++it;
-            mbar_arrive_expect_tx(&sh.full[s], A_BYTES + b_bytes);
             uint8_t* a_dst = smem + s * A_BYTES;
-            uint8_t* b_dst = smem + NS * A_BYTES + s * B_BYTES;
-            tma_load_2d(a_dst, tmA, &sh.full[s], (int32_t)(kb * BK), (int32_t)m0);
-            if (p.b_major == FP8_B_KMAJOR) {
-                tma_load_2d(b_dst, tmB, &sh.full[s], (int32_t)(kb * BK), brow);
+            uint8_t* b_dst = smem + NS * A_BYTES + s * T::B_BYTES;
+            if (PAIR) {
+                // both CTAs' bytes count on the even CTA's barrier
+                const uint32_t bar = mapa_shared(smem_u32(&sh.full[s]), 0);
+                if (rank == 0) mbar_arrive_expect_tx(&sh.full[s], 2 * (A_BYTES + b_bytes));
+                tma_load_2d_pair(a_dst, tmA, bar, (int32_t)(kb * BK), (int32_t)m0);
+                if (p.b_major == FP8_B_KMAJOR)
+                    tma_load_2d_pair(b_dst, tmB, bar, (int32_t)(kb * BK), brow);
+                else
+                    tma_load_2d_pair(b_dst, tmB, bar, (int32_t)(n0 + rank * 128),
+                                     (int32_t)(kb * BK));
             } else {
-                tma_load_2d(b_dst, tmB, &sh.full[s], (int32_t)n0, (int32_t)(kb * BK));
-                if (n_valid > 128)
-                    tma_load_2d(b_dst + 128 * BK, tmB, &sh.full[s], (int32_t)(n0 + 128),
-                                (int32_t)(kb * BK));
+                mbar_arrive_expect_tx(&sh.full[s], A_BYTES + b_bytes);
+                tma_load_2d(a_dst, tmA, &sh.full[s], (int32_t)(kb * BK), (int32_t)m0);
+                if (p.b_major == FP8_B_KMAJOR) {
+                    tma_load_2d(b_dst, tmB, &sh.full[s], (int32_t)(kb * BK), brow);
+                } else {
+                    tma_load_2d(b_dst, tmB, &sh.full[s], (int32_t)n0, (int32_t)(kb * BK));
+                    if (n_valid > 128)
+                        tma_load_2d(b_dst + 128 * BK, tmB, &sh.full[s], (int32_t)(n0 + 128),
+                                    (int32_t)(kb * BK));
+                }
             }
         }
     }
-    // every copy issued lands before the CTA exits
+    // every copy issued lands before the CTA exits (a pair's all count on the
+    // even CTA's barriers; the odd CTA stays until the closing cluster barrier)
+    if (PAIR && rank != 0) return;
 #pragma unroll
     for (int s = 0; s < NS; ++s) {
         const int64_t count = it > s ? (it - s + NS - 1) / NS : 0;
@@ -238,25 +316,33 @@ __device__ void mx_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, cons
 // idle.  The loop therefore waits for the next stage before issuing the
 // current stage's last MMA, so the barrier latency hides behind the MMAs
 // still executing, and it spins rather than suspends on barriers.
+template <bool PAIR>
 __device__ void mx_mma(const MxParams& p, uint8_t* smem, MxShared& sh, int64_t nmb, int64_t nnb,
                        int64_t nkb)
 {
+    using T = MxTiling<PAIR>;
+    constexpr int NS = T::NS;
     volatile int* abort = &sh.abort;
     const uint32_t a_base = smem_u32(smem);
     const uint32_t b_base = a_base + NS * A_BYTES;
-    const uint32_t sf_base = b_base + NS * B_BYTES;
+    const uint32_t sf_base = b_base + NS * T::B_BYTES;
     const uint32_t tmem = sh.tmem_base;
     const int64_t ntiles = nmb * nnb;
     uint32_t it = 0;          // K-blocks consumed so far (stage it % NS, round it / NS)
     uint32_t tcount = 0;
     bool ok = true;
-    for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+    int64_t first, stride;
+    mx_unit_range<PAIR>(first, stride);
+    for (int64_t tile = first; ok && tile < ntiles; tile += stride) {
         int64_t mb, nb;
         gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
-        if (p.group_offsets && find_group(sh.off, p.G, mb * BM) < 0) continue;
+        if (!PAIR && p.group_offsets && find_group(sh.off, p.G, mb * BM) < 0) continue;
         const int64_t n0 = nb * BN;
         const int64_t n_valid = (p.N - n0 < BN) ? (p.N - n0) : BN;
-        const uint32_t idesc = idesc_mx_e4m3(BM, (uint32_t)n_valid, (uint32_t)p.b_major);
+        // a pair's MMA always spans 256 columns (a B tail is zero-filled)
+        const uint32_t idesc = idesc_mx_e4m3((uint32_t)T::TILE_M,
+                                             PAIR ? (uint32_t)BN : (uint32_t)n_valid,
+                                             (uint32_t)p.b_major);
         // the epilogue has read the previous tile's accumulator
         ok = mbar_wait_spin(&sh.acc_empty, (tcount & 1u) ^ 1u, abort, p.timeout_ns) &&
              mbar_wait_spin(&sh.full[it % NS], (it / NS) & 1u, abort, p.timeout_ns);
@@ -265,12 +351,18 @@ __device__ void mx_mma(const MxParams& p, uint8_t* smem, MxShared& sh, int64_t n
             const uint32_t s = it % NS;
             tc_fence_after();
             const uint32_t a_addr = a_base + s * A_BYTES;
-            const uint32_t b_addr = b_base + s * B_BYTES;
+            const uint32_t b_addr = b_base + s * T::B_BYTES;
             const uint32_t sf_addr = sf_base + s * SF_BYTES;
             const uint32_t sfa = tmem + SF_COL0 + s * SF_SLOT_COLS;
-            tmem_cp_32x128b_x4(sfa, sf_addr);                               // SFA, rows 0-127
-            tmem_cp_32x128b_x4(sfa + SFB_OFF, sf_addr + SFA_BYTES);         // SFB, columns 0-127
-            tmem_cp_32x128b_x4(sfa + SFB_OFF + 4, sf_addr + SFA_BYTES + 512);   // columns 128-255
+            if (PAIR) {
+                tmem_cp_32x128b_x4_pair(sfa, sf_addr);
+                tmem_cp_32x128b_x4_pair(sfa + SFB_OFF, sf_addr + SFA_BYTES);
+                tmem_cp_32x128b_x4_pair(sfa + SFB_OFF + 4, sf_addr + SFA_BYTES + 512);
+            } else {
+                tmem_cp_32x128b_x4(sfa, sf_addr);                               // SFA, rows 0-127
+                tmem_cp_32x128b_x4(sfa + SFB_OFF, sf_addr + SFA_BYTES);         // SFB, columns 0-127
+                tmem_cp_32x128b_x4(sfa + SFB_OFF + 4, sf_addr + SFA_BYTES + 512);   // columns 128-255
+            }
 #pragma unroll
             for (int k = 0; k < BK / 32; ++k) {
                 if (k == BK / 32 - 1 && kb + 1 < nkb) {
@@ -285,32 +377,47 @@ __device__ void mx_mma(const MxParams& p, uint8_t* smem, MxShared& sh, int64_t n
                 const uint64_t bdesc = (p.b_major == FP8_B_KMAJOR)
                                            ? smem_desc_sw128(b_addr + k * 32, 16, 1024)
                                            : smem_desc_sw128(b_addr + k * 32 * 128, 128 * BK, 1024);
-                mma_mxf8(tmem, adesc, bdesc, idesc, sfa, sfa + SFB_OFF, (kb | k) ? 1u : 0u);
+                const uint32_t acc = (kb | k) ? 1u : 0u;
+                if (PAIR)
+                    mma_mxf8_pair(tmem, adesc, bdesc, idesc, sfa, sfa + SFB_OFF, acc);
+                else
+                    mma_mxf8(tmem, adesc, bdesc, idesc, sfa, sfa + SFB_OFF, acc);
             }
-            mma_commit(&sh.empty[s]);        // stage and scale slot free once these are done
+            // stage and scale slot free once these are done (in both CTAs)
+            if (PAIR)
+                mma_commit_pair(&sh.empty[s], 3);
+            else
+                mma_commit(&sh.empty[s]);
             if (!ok) break;
         }
         if (!ok) break;
-        mma_commit(&sh.acc_full);            // the tile's sum is complete
+        // the tile's sum is complete
+        if (PAIR)
+            mma_commit_pair(&sh.acc_full, 3);
+        else
+            mma_commit(&sh.acc_full);
         ++tcount;
     }
-    mma_commit(&sh.drain);
+    if (PAIR)
+        mma_commit_pair(&sh.drain, 1);
+    else
+        mma_commit(&sh.drain);
     mbar_wait_drain(&sh.drain, 0, p.timeout_ns);
 }
 
 // Scales of K-block kb handled by scale-writer thread t (0..127): row t of
-// the tile's A block and columns t, t + 128 of its B block; 1 outside the
-// matrix.
+// the CTA's A block and columns t, t + 128 of the tile's B block; 1 outside
+// the matrix or the tile's group.
 struct SfRegs {
     float a;
     float b[2];
 };
 
-__device__ __forceinline__ void load_sf(const MxParams& p, int g, int64_t m0, int64_t n0, int64_t kb,
-                                        int64_t nkb, int t, SfRegs& r)
+__device__ __forceinline__ void load_sf(const MxParams& p, int g, int64_t m0, int64_t m_end,
+                                        int64_t n0, int64_t kb, int64_t nkb, int t, SfRegs& r)
 {
     const int64_t m = m0 + t;
-    r.a = m < p.M ? __ldg(p.sA + kb * p.M + m) : 1.0f;
+    r.a = m < m_end ? __ldg(p.sA + kb * p.M + m) : 1.0f;
     const int64_t nnb128 = p.N / 128;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -332,31 +439,34 @@ __device__ __forceinline__ void load_sf(const MxParams& p, int g, int64_t m0, in
 // line i % 32, word i / 32.
 __device__ __forceinline__ uint32_t sf_offset(int i) { return 16u * (uint32_t)(i & 31) + 4u * (uint32_t)(i >> 5); }
 
+template <bool PAIR>
 __device__ void mx_scale_writer(const MxParams& p, uint8_t* smem, MxShared& sh, int64_t nmb,
                                 int64_t nnb, int64_t nkb, int warp, int lane)
 {
+    using T = MxTiling<PAIR>;
+    constexpr int NS = T::NS;
     volatile int* abort = &sh.abort;
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
     const int t = (warp - FIRST_SF_WARP) * 32 + lane;          // 0..127
-    uint8_t* sf_base = smem + NS * (A_BYTES + B_BYTES);
+    uint8_t* sf_base = smem + NS * (A_BYTES + T::B_BYTES);
     const uint32_t off_a = sf_offset(t);
     const uint32_t off_b0 = SFA_BYTES + sf_offset(t);
     const uint32_t off_b1 = SFA_BYTES + 512 + sf_offset(t);
     int64_t it = 0;
     bool ok = true, bad = false;
-    for (int64_t tile = blockIdx.x; ok && tile < nmb * nnb; tile += gridDim.x) {
+    int64_t first, stride;
+    mx_unit_range<PAIR>(first, stride);
+    for (int64_t tile = first; ok && tile < nmb * nnb; tile += stride) {
         int64_t mb, nb;
         gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
-        const int64_t m0 = mb * BM, n0 = nb * BN;
-        int g = 0;
-        if (p.group_offsets) {
-            g = find_group(sh.off, p.G, m0);
-            if (g < 0) continue;
-        }
+        TileRows tr;
+        if (!mx_tile_rows<PAIR>(p, sh, mb, rank, tr)) continue;
+        const int64_t n0 = nb * BN;
         // SF_AHEAD K-blocks of scale loads in flight per thread
         SfRegs ring[SF_AHEAD];
 #pragma unroll
         for (int u = 0; u < SF_AHEAD; ++u)
-            if (u < nkb) load_sf(p, g, m0, n0, u, nkb, t, ring[u]);
+            if (u < nkb) load_sf(p, tr.g, tr.m0, tr.m_end, n0, u, nkb, t, ring[u]);
         for (int64_t kb0 = 0; ok && kb0 < nkb; kb0 += SF_AHEAD) {
 #pragma unroll
             for (int u = 0; u < SF_AHEAD; ++u) {
@@ -365,7 +475,8 @@ __device__ void mx_scale_writer(const MxParams& p, uint8_t* smem, MxShared& sh, 
                     const uint32_t wa = ue8m0_x4(ring[u].a, bad);
                     const uint32_t wb0 = ue8m0_x4(ring[u].b[0], bad);
                     const uint32_t wb1 = ue8m0_x4(ring[u].b[1], bad);
-                    if (kb + SF_AHEAD < nkb) load_sf(p, g, m0, n0, kb + SF_AHEAD, nkb, t, ring[u]);
+                    if (kb + SF_AHEAD < nkb)
+                        load_sf(p, tr.g, tr.m0, tr.m_end, n0, kb + SF_AHEAD, nkb, t, ring[u]);
                     const int s = (int)(it % NS);
                     const uint32_t ph = (uint32_t)((it / NS) & 1);
                     // the copies and MMAs that last read this stage have completed
@@ -377,7 +488,12 @@ __device__ void mx_scale_writer(const MxParams& p, uint8_t* smem, MxShared& sh, 
                         *reinterpret_cast<uint32_t*>(sf + off_b1) = wb1;
                         fence_proxy_async_smem();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(&sh.full[s]);
+                        if (lane == 0) {
+                            if (PAIR)   // the even CTA's MMA thread copies both CTAs' blocks
+                                mbar_arrive_cluster(mapa_shared(smem_u32(&sh.full[s]), 0));
+                            else
+                                mbar_arrive(&sh.full[s]);
+                        }
                     } else {
                         ok = false;
                     }
@@ -388,25 +504,31 @@ __device__ void mx_scale_writer(const MxParams& p, uint8_t* smem, MxShared& sh, 
     if (__any_sync(0xffffffffu, bad) && lane == 0) report_error(FP8_ERR_VALUE);
 }
 
+template <bool PAIR>
 __device__ void mx_epilogue(const MxParams& p, MxShared& sh, int64_t nmb, int64_t nnb, int warp,
                             int lane)
 {
     volatile int* abort = &sh.abort;
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
     const int ew = warp - FIRST_EPI_WARP;       // 0..7
     const int q = warp & 3;
     const int col0 = (ew >> 2) * 128;
     const int row = q * 32 + lane;
     const uint32_t taddr0 = sh.tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)col0;
     uint32_t tcount = 0;
-    for (int64_t tile = blockIdx.x; tile < nmb * nnb; tile += gridDim.x) {
+    int64_t first, stride;
+    mx_unit_range<PAIR>(first, stride);
+    for (int64_t tile = first; tile < nmb * nnb; tile += stride) {
         int64_t mb, nb;
         gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
-        if (p.group_offsets && find_group(sh.off, p.G, mb * BM) < 0) continue;
+        TileRows tr;
+        if (!mx_tile_rows<PAIR>(p, sh, mb, rank, tr)) continue;
         const uint32_t tph = tcount++ & 1u;
-        const int64_t m = mb * BM + row;
+        const int64_t m = tr.m0 + row;
         const int64_t n0 = nb * BN + col0;
-        const bool active = n0 < p.N;           // warp-uniform
-        const bool row_ok = m < p.M;
+        // warp-uniform: columns inside N and this CTA's rows inside the group
+        const bool active = n0 < p.N && tr.m0 < tr.m_end;
+        const bool row_ok = m < tr.m_end;
         if (!warp_wait(&sh.acc_full, tph, abort, p.timeout_ns, lane)) break;
         tc_fence_after();
 #pragma unroll 1
@@ -419,7 +541,12 @@ __device__ void mx_epilogue(const MxParams& p, MxShared& sh, int64_t nmb, int64_
             if (c == 3) {                        // accumulator no longer needed
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sh.acc_empty);
+                if (lane == 0) {
+                    if (PAIR)   // the even CTA's MMA waits for both CTAs' epilogues
+                        mbar_arrive_cluster(mapa_shared(smem_u32(&sh.acc_empty), 0));
+                    else
+                        mbar_arrive(&sh.acc_empty);
+                }
             }
             if (!(active && row_ok)) continue;
             if (p.out_dtype == FP8_OUT_BF16) {
@@ -444,28 +571,32 @@ __device__ void mx_epilogue(const MxParams& p, MxShared& sh, int64_t nmb, int64_
     }
 }
 
+template <bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_fp8_gemm_mx(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const MxParams p)
 {
+    using T = MxTiling<PAIR>;
     extern __shared__ uint8_t smem_raw[];
     __shared__ MxShared sh;
+    // same 1024-byte-aligned offset in both CTAs of a pair
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int64_t nmb = (p.M + BM - 1) / BM;
     const int64_t nnb = (p.N + BN - 1) / BN;
     const int64_t nkb = p.K / BK;
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < NS; ++s) {
-            mbar_init(&sh.full[s], 1 + NUM_SF_WARPS);
+        for (int s = 0; s < T::NS; ++s) {
+            // the TMA bytes' arrive plus every scale warp (of both CTAs of a pair)
+            mbar_init(&sh.full[s], 1 + (PAIR ? 2 : 1) * NUM_SF_WARPS);
             mbar_init(&sh.empty[s], 1);
         }
         mbar_init(&sh.acc_full, 1);
-        mbar_init(&sh.acc_empty, NUM_EPI_WARPS);
+        mbar_init(&sh.acc_empty, (PAIR ? 2 : 1) * NUM_EPI_WARPS);
         mbar_init(&sh.drain, 1);
         sh.abort = 0;
         sh.bad = 0;
@@ -474,13 +605,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tma_prefetch_desc(&tmB);
     }
     if (warp == 2) {
-        tmem_alloc(&sh.tmem_base, TMEM_COLS);
-        tmem_relinquish();
+        if (PAIR) {
+            tmem_alloc_pair(&sh.tmem_base, TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(&sh.tmem_base, TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     if (p.group_offsets)
         for (int i = threadIdx.x; i <= p.G; i += NUM_THREADS) sh.off[i] = p.group_offsets[i];
+    // barrier inits and the TMEM address visible to the peer CTA before use
     tc_fence_before();
-    __syncthreads();
+    if (PAIR)
+        cluster_sync();
+    else
+        __syncthreads();
     tc_fence_after();
     if (threadIdx.x == 0) {
         bool bad = false;
@@ -492,40 +632,92 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         sh.bad = bad ? 1 : 0;
     }
     __syncthreads();
+    if (PAIR && p.group_offsets && !sh.bad && warp == 0)
+        pair_block_offsets(sh.off, sh.poff, p.G, lane);
+    __syncthreads();
+    const int64_t nmb = (PAIR && p.group_offsets) ? (int64_t)sh.poff[p.G]
+                                                  : (p.M + T::TILE_M - 1) / T::TILE_M;
 
     if (sh.bad) {
         // malformed offsets: nothing is loaded, multiplied or written
     } else if (warp == 0) {
-        if (lane == 0) mx_producer(&tmA, &tmB, p, smem, sh, nmb, nnb, nkb);
+        if (lane == 0) mx_producer<PAIR>(&tmA, &tmB, p, smem, sh, nmb, nnb, nkb);
         __syncwarp();
     } else if (warp == 1) {
-        if (lane == 0) mx_mma(p, smem, sh, nmb, nnb, nkb);
+        if (lane == 0 && rank == 0) mx_mma<PAIR>(p, smem, sh, nmb, nnb, nkb);
         __syncwarp();
     } else if (warp >= FIRST_SF_WARP && warp < FIRST_SF_WARP + NUM_SF_WARPS) {
-        mx_scale_writer(p, smem, sh, nmb, nnb, nkb, warp, lane);
+        mx_scale_writer<PAIR>(p, smem, sh, nmb, nnb, nkb, warp, lane);
     } else if (warp >= FIRST_EPI_WARP) {
-        mx_epilogue(p, sh, nmb, nnb, warp, lane);
+        mx_epilogue<PAIR>(p, sh, nmb, nnb, warp, lane);
     }
     tc_fence_before();
-    __syncthreads();
+    if (PAIR)
+        cluster_sync();
+    else
+        __syncthreads();
     tc_fence_after();
-    if (warp == 2) tmem_dealloc(sh.tmem_base, TMEM_COLS);
+    if (warp == 2) {
+        if (PAIR)
+            tmem_dealloc_pair(sh.tmem_base, TMEM_COLS);
+        else
+            tmem_dealloc(sh.tmem_base, TMEM_COLS);
+    }
 }
 
-bool ensure_mx_smem_attr()
+cudaLaunchConfig_t mx_pair_config(unsigned clusters, cudaStream_t st, cudaLaunchAttribute* attr)
 {
-    static bool done[64] = {};
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * clusters, 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = DYN_SMEM;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cfg;
+}
+
+// Once per device: shared-memory opt-in for both kernels and the number of
+// CTA pairs that fit at once (0: pairs unavailable, single CTAs are used).
+struct MxDeviceSetup {
+    bool ok = false;
+    int pair_clusters = 0;
+};
+
+MxDeviceSetup mx_device_setup()
+{
+    static MxDeviceSetup done[64];
+    static bool tried[64] = {};
     static std::mutex mu;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MxDeviceSetup{};
     std::lock_guard<std::mutex> lk(mu);
-    if (!done[dev]) {
-        if (cudaFuncSetAttribute(k_fp8_gemm_mx, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)DYN_SMEM) != cudaSuccess)
-            return false;
-        done[dev] = true;
+    if (!tried[dev]) {
+        tried[dev] = true;
+        MxDeviceSetup r;
+        r.ok = cudaFuncSetAttribute(k_fp8_gemm_mx<false>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)DYN_SMEM) == cudaSuccess &&
+               cudaFuncSetAttribute(k_fp8_gemm_mx<true>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)DYN_SMEM) == cudaSuccess;
+        if (r.ok) {
+            cudaLaunchAttribute attr[1];
+            const cudaLaunchConfig_t cfg = mx_pair_config((unsigned)device_sm_count(), nullptr, attr);
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, k_fp8_gemm_mx<true>, &cfg) != cudaSuccess) {
+                n = 0;
+                (void)cudaGetLastError();
+            }
+            r.pair_clusters = n;
+        }
+        done[dev] = r;
     }
-    return true;
+    return done[dev];
 }
 
 }  // namespace
@@ -536,8 +728,11 @@ int launch_blockscaled_gemm_mx(const uint8_t* A, const float* sA, const uint8_t*
                                int64_t ldd, cudaStream_t st)
 {
     if (M == 0) return FP8_OK;
+    const MxDeviceSetup setup = mx_device_setup();
+    if (!setup.ok) return FP8_ERR_LAUNCH;
+    const bool pair = setup.pair_clusters > 0;
     CUtensorMap tmA, tmB;
-    const int b_box_rows = N >= BN ? BN : (int)N;
+    const int b_box_rows = pair ? 128 : (N >= BN ? BN : (int)N);
     if (!make_map(&tmA, A, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, BM)) return FP8_ERR_LAUNCH;
     bool okB;
     if (b_major == FP8_B_KMAJOR) {
@@ -546,7 +741,7 @@ int launch_blockscaled_gemm_mx(const uint8_t* A, const float* sA, const uint8_t*
     } else {
         okB = make_map(&tmB, B, (uint64_t)N, (uint64_t)K, (uint64_t)N, 128, BK);
     }
-    if (!okB || !ensure_mx_smem_attr()) return FP8_ERR_LAUNCH;
+    if (!okB) return FP8_ERR_LAUNCH;
 
     MxParams p;
     p.sA = sA;
@@ -564,10 +759,21 @@ int launch_blockscaled_gemm_mx(const uint8_t* A, const float* sA, const uint8_t*
     p.b_box_rows = b_box_rows;
     p.timeout_ns = wait_timeout_ns();
 
-    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int64_t nnb = (N + BN - 1) / BN;
+    if (pair) {
+        // grouped: each group adds at most one partly idle 256-row block
+        const int64_t tiles = ((M + 255) / 256 + (group_offsets ? G : 0)) * nnb;
+        const int64_t clusters = tiles < setup.pair_clusters ? tiles : setup.pair_clusters;
+        cudaLaunchAttribute attr[1];
+        const cudaLaunchConfig_t cfg = mx_pair_config((unsigned)clusters, st, attr);
+        return cudaLaunchKernelEx(&cfg, k_fp8_gemm_mx<true>, tmA, tmB, p) == cudaSuccess
+                   ? FP8_OK
+                   : FP8_ERR_LAUNCH;
+    }
+    const int64_t tiles = ((M + BM - 1) / BM) * nnb;
     const int sms = device_sm_count();
     const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
-    k_fp8_gemm_mx<<<grid, NUM_THREADS, DYN_SMEM, st>>>(tmA, tmB, p);
+    k_fp8_gemm_mx<false><<<grid, NUM_THREADS, DYN_SMEM, st>>>(tmA, tmB, p);
     return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_LAUNCH;
 }
 
