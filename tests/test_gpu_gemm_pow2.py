@@ -89,6 +89,20 @@ def test_pow2_gemm_reports_non_power_of_two_scale():
     assert fg.fp8_get_status() == fg.FP8_OK
 
 
+@pytest.mark.parametrize("row", [5, 200])
+def test_pow2_gemm_reports_bad_scale_in_either_half_of_a_pair_tile(row):
+    """Rows 0-127 and 128-255 of a 256-row tile are scaled by different CTAs;
+    a non-power-of-two scale in either is reported."""
+    M, N, K = 256, 256, 256
+    qa, sa, qw, sw = _operands(M, N, K, seed=17)
+    sa = sa.copy()
+    sa[1, row] = np.float32(3.0)
+    D = torch.empty((M, N), dtype=torch.float32, device=dev())
+    fg.fp8_blockscaled_gemm_pow2(to_dev(qa), to_dev(sa), to_dev(qw), to_dev(sw), D)
+    assert fg.fp8_get_status() == fg.FP8_ERR_VALUE
+    assert fg.fp8_get_status() == fg.FP8_OK
+
+
 def _pow2(s):
     """Nearest power of two of each positive scale (test input construction)."""
     return np.exp2(np.round(np.log2(s))).astype(np.float32)
