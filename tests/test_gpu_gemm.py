@@ -57,7 +57,7 @@ CASES = [
     (384, 640, 384, fg.B_KMAJOR, 1),
     (384, 640, 256, fg.B_MNMAJOR, 128),
     (300, 640, 256, fg.B_KMAJOR, 128),
-    # per-column B scales, N an odd number of 128-column halves (last tile half empty)
+    # per-column B scales: N = 896 leaves the last 256-wide tile half empty
     (256, 896, 512, fg.B_KMAJOR, 1),
     (300, 1792, 640, fg.B_KMAJOR, 1),
 ]
