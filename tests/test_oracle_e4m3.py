@@ -1,8 +1,9 @@
 """Pins of the oracle's E4M3 codec against things other than itself.
 
 The pages fix E4M3 "on all tensors" (4 exponent bits, 3 mantissa bits) for
-Fprop, Dgrad and Wgrad (Mixed precision framework, Figure 6); rounding to
-nearest-even and saturation are this build's readings R2.
+Fprop, Dgrad and Wgrad (Mixed precision framework, Figure 6); the pages do
+not state the rounding, so the oracle rounds to nearest-even and saturates at
++-448 (reading R2 in the header of oracle/fp8_oracle.c).
 
 Independent references used here:
   * torch's own float8_e4m3fn type (a library implementation of OCP E4M3FN):
