@@ -24,7 +24,7 @@
  *   - Integral power-of-2 scaling factors are used for some activations
  *     (Linear after attention; activation gradient before MoE down-proj).
  *
- * Readings where the pages are silent (each restated in the design doc):
+ * Readings where the pages are silent:
  *   R1  stored scale s is the dequantisation multiplier amax/448; values are
  *       encoded as E(fl32(x * fl32(448/amax))).  All scale arithmetic is
  *       correctly rounded FP32 (the precision of the stored scale).

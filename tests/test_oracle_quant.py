@@ -9,6 +9,10 @@ integral powers of 2.  The checks below are closed forms, invariants,
 planted-layout cases and exact special cases -- none re-types the oracle's
 scale formula.
 """
+import bisect
+import math
+from fractions import Fraction
+
 import numpy as np
 import pytest
 import torch
@@ -31,6 +35,53 @@ def _bits(x32):
 
 def _from_bits(b):
     return (b.astype(np.uint32) << 16).view(np.float32)
+
+
+# ---------------------------------------------------------------- exact arithmetic
+# Correct rounding written out on rationals: no float operation decides a
+# result, so these checks pin the oracle's FP32 arithmetic itself.
+
+def fl32(fr: Fraction) -> Fraction:
+    """The FP32 value nearest to the positive rational fr, ties to the even
+    significand (normal FP32 range)."""
+    assert fr > 0
+    e = fr.numerator.bit_length() - fr.denominator.bit_length()   # 2^e <= fr < 2^(e+2)
+    if Fraction(2) ** e > fr:
+        e -= 1
+    elif Fraction(2) ** (e + 1) <= fr:
+        e += 1
+    assert -126 <= e <= 127
+    ulp = Fraction(2) ** (e - 23)
+    n = math.floor(fr / ulp)                  # 2^23 <= n < 2^24
+    rem = fr / ulp - n
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    return n * ulp
+
+
+def fl32_signed(fr: Fraction) -> Fraction:
+    return fl32(fr) if fr > 0 else -fl32(-fr)
+
+
+# non-negative finite E4M3 values in code order (torch's float8_e4m3fn table)
+_POS = [Fraction(float(TAB[c])) for c in range(0x7F)]
+
+
+def e4m3_nearest(y: Fraction, negative: bool) -> int:
+    """Code of the E4M3 value nearest to y (ties to the even code, |y| >= 448
+    saturating to 448), with the sign bit of the input."""
+    a = abs(y)
+    sign = 0x80 if negative else 0
+    if a >= 448:
+        return sign | 0x7E
+    hi = bisect.bisect_left(_POS, a)
+    if _POS[hi] == a:
+        return sign | hi
+    lo = hi - 1
+    dlo, dhi = a - _POS[lo], _POS[hi] - a
+    if dlo < dhi or (dlo == dhi and lo % 2 == 0):
+        return sign | lo
+    return sign | hi
 
 
 # ---------------------------------------------------------------- layout pins
@@ -99,6 +150,124 @@ def test_128x128_planted_block_maxima_fix_scale_layout():
             assert q[nb * 128 + (nb * 37 + kb * 11) % 128, kb * 128 + (nb * 5 + kb * 71) % 128] == 0xFE
 
 
+# ---------------------------------------------------------------- exact scale and codes
+# Reading R1: s = fl32(amax/448) is stored and the codes are
+# E(fl32(x * fl32(448/amax))).  Written out on rationals; the groups hold
+# max-abs values that are not powers of two (where 1/448 and 448/amax are
+# inexact) and elements planted within a few FP32 ulps of a midpoint between
+# two E4M3 values, so that a product formed any other way -- x/s, or
+# x * fl32(1/s) -- rounds to the neighbouring code.
+
+def _ulp32(v: Fraction) -> Fraction:
+    e = v.numerator.bit_length() - v.denominator.bit_length()
+    if Fraction(2) ** e > v:
+        e -= 1
+    elif Fraction(2) ** (e + 1) <= v:
+        e += 1
+    return Fraction(2) ** (e - 23)
+
+
+def _f32(v: Fraction):
+    """v as an np.float32 if it is an FP32 value, else None."""
+    f = np.float32(float(v))
+    return f if Fraction(float(f)) == v else None
+
+
+def _non_pow2_amax(rng):
+    while True:
+        a = np.float32(rng.uniform(1.0, 2.0) * 2.0 ** int(rng.integers(-20, 21)))
+        if math.frexp(float(a))[0] != 0.5:
+            return a
+
+
+def _planted_values(rng, amax, n, n_planted):
+    """n values below amax in magnitude: random ones, and n_planted placed at
+    E4M3 rounding midpoints of the scaled space, alternately chosen where
+    fl32(x/s) and where fl32(x*fl32(1/s)) round to another code than
+    fl32(x*inv)."""
+    A = Fraction(float(amax))
+    inv, s = fl32(448 / A), fl32(A / 448)
+    r = fl32(1 / s)
+    out = (rng.uniform(2.0 ** -12, 1.0, n) * float(amax)).astype(np.float32)
+    for i in range(n_planted):
+        c = int(rng.integers(8, 0x7D))                    # normal codes c, c+1
+        mid = (_POS[c] + _POS[c + 1]) / 2
+        x0 = fl32(mid / inv)
+        pick = _f32(x0)
+        for k in (0, 1, -1, 2, -2, 3, -3, 4, -4):
+            x = _f32(x0 + k * _ulp32(x0))
+            if x is None:
+                continue
+            X = Fraction(float(x))
+            good = e4m3_nearest(fl32(X * inv), False)
+            other = fl32(X / s) if i % 2 == 0 else fl32(X * r)
+            if e4m3_nearest(other, False) != good:
+                pick = x
+                break
+        out[i] = pick
+    out *= np.where(rng.integers(0, 2, n) == 1, -1, 1).astype(np.float32)
+    return out
+
+
+def _expected_group(vals):
+    """(scale, codes) of one group from the definition, on rationals."""
+    A = max(abs(Fraction(float(v))) for v in vals)
+    inv = fl32(448 / A)
+    codes = [e4m3_nearest(fl32_signed(Fraction(float(v)) * inv), bool(np.signbit(v)))
+             for v in vals]
+    return fl32(A / 448), np.array(codes, np.uint8)
+
+
+def _planted_group(rng, n=128, n_planted=48):
+    amax = _non_pow2_amax(rng)
+    g = _planted_values(rng, amax, n, n_planted)
+    g[int(rng.integers(n_planted, n))] = amax * (1 if rng.integers(0, 2) else -1)
+    return g
+
+
+def test_fp32_scale_and_codes_are_the_correctly_rounded_definition_1x128():
+    rng = np.random.default_rng(21)
+    M, K = 8, 512
+    x = np.stack([np.concatenate([_planted_group(rng) for _ in range(K // 128)])
+                  for _ in range(M)]).astype(np.float32)
+    q, s = oracle.quant_act_1x128(x)
+    for m in range(M):
+        for kb in range(K // 128):
+            want_s, want_q = _expected_group(x[m, kb * 128:(kb + 1) * 128])
+            assert Fraction(float(s[kb, m])) == want_s, (m, kb)
+            assert np.array_equal(q[m, kb * 128:(kb + 1) * 128], want_q), (m, kb)
+
+
+def test_fp32_scale_and_codes_are_the_correctly_rounded_definition_128x1():
+    rng = np.random.default_rng(22)
+    T, C = 256, 16
+    x = np.stack([np.concatenate([_planted_group(rng) for _ in range(T // 128)])
+                  for _ in range(C)], axis=1).astype(np.float32)      # [T, C]
+    qT, s = oracle.quant_act_128x1(x)
+    for tb in range(T // 128):
+        for c in range(C):
+            want_s, want_q = _expected_group(x[tb * 128:(tb + 1) * 128, c])
+            assert Fraction(float(s[tb, c])) == want_s, (tb, c)
+            assert np.array_equal(qT[c, tb * 128:(tb + 1) * 128], want_q), (tb, c)
+
+
+def test_fp32_scale_and_codes_are_the_correctly_rounded_definition_128x128():
+    rng = np.random.default_rng(23)
+    N, K = 128, 256
+    w = np.empty((N, K), np.float32)
+    for kb in range(K // 128):
+        amax = _non_pow2_amax(rng)
+        blk = _planted_values(rng, amax, 128 * 128, 160)
+        blk[int(rng.integers(160, 128 * 128))] = -amax
+        w[:, kb * 128:(kb + 1) * 128] = rng.permutation(blk).reshape(128, 128)
+    q, s = oracle.quant_w_128x128(w)
+    for kb in range(K // 128):
+        blk = w[:, kb * 128:(kb + 1) * 128]
+        want_s, want_q = _expected_group(blk.reshape(-1))
+        assert Fraction(float(s[0, kb])) == want_s, kb
+        assert np.array_equal(q[:, kb * 128:(kb + 1) * 128].reshape(-1), want_q), kb
+
+
 # ---------------------------------------------------------------- invariants
 
 def _groups_1x128(a):
@@ -120,10 +289,11 @@ def test_every_nonzero_group_has_a_448_code_and_bounded_round_trip(dtype):
     assert np.array_equal(has448, amax > 0)
     # zero group: scale 1, codes +-0
     assert s[1, 3] == 1.0 and np.all((g[3, 1] & 0x7F) == 0)
-    # scale within one FP32 rounding of amax/448 (closed form, not the formula)
+    # the stored scale is amax/448 correctly rounded to FP32 (exact rationals)
     nz = amax > 0
     sv = s.T.astype(np.float64)
-    assert np.all(np.abs(sv[nz] * 448.0 - amax[nz]) <= amax[nz] * 2.0 ** -23)
+    want = [fl32(Fraction(float(a)) / 448) for a in amax[nz]]
+    assert [Fraction(float(v)) for v in sv[nz]] == want
     # round trip: relative error <= 2^-4 (3 mantissa bits, RNE) in the normal range
     deq = dec(g) * sv[:, :, None]
     r = np.abs(xv) / sv[:, :, None]
