@@ -4,11 +4,14 @@
                     [--impl ours|reference]
 
 A step is one pass of the hot path over one batch of synthetic input on the
-chosen workload (default: the dense-MLP Fprop shape, X[4096,7168] and
-W[18432,7168] in BF16): 1x128 activation quantization, 128x128 weight
-quantization and the block-scaled FP8 GEMM with FP32 promotion per 128-K
-block, BF16 output.  Other workloads (--workload dgrad|wgrad|wgrad_pow2|moe|
-pr1) run the other passes of the Linear the same way.
+chosen workload.  The default is the largest configuration by FLOPs, the MoE
+grouped Fprop: 16384 tokens X[16384,7168] in BF16, top-8 routing drawn from
+a Zipf(1.1) law over 32 experts W_e[2048,7168]; one step is the 1x128
+activation quantization, the FP8 dispatch of the token rows into
+expert-contiguous groups padded to 128 rows, the 128x128 weight
+quantization and the grouped block-scaled FP8 GEMM with FP32 promotion per
+128-K block, BF16 output.  Other workloads (--workload fprop|dgrad|wgrad|
+wgrad_pow2|pr1|...) run the other passes of the Linear the same way.
 
 The metric is FP8 block-scaled GEMM throughput: 2*M*N*K algorithmic FLOPs
 per step divided by the device time of the whole step (quantizers included),
@@ -19,8 +22,14 @@ collective); time is the max over ranks.
 The JSON line also carries
   roofline      the GEMM kernel's achieved TFLOP/s (CUDA events around its
                 launches in the timed region) against the FP8 peak derived
-                from the measured BF16 peak x 2 (nominal FP8/BF16 ratio), and
-                the quantizers' GB/s against the measured HBM copy bandwidth;
+                from the measured BF16 peak x 2 (nominal FP8/BF16 ratio):
+                the burst figure when the sampled SM clock stayed at its
+                maximum with no power-cap event, else the sustained one; the
+                same rate also against the tensor cores' clock-scaled
+                ceiling (148 SMs x 16384 FP8 FLOP/clk x sampled SM clock) and
+                the 4.5 PFLOP/s dense FP8 specification; the quantizers'
+                GB/s against the measured HBM copy bandwidth and the 8 TB/s
+                specification;
   cpu_baseline  the CPU oracle timed on this host on a bounded sample of the
                 same workload (rank 0, N = 1 only), extrapolated to a step;
   e2e           the same metric through the C ABI with the inputs copied from
@@ -59,6 +68,49 @@ def measured_peaks():
                     source="measured")
     except Exception:
         return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+SM_COUNT = 148
+FP8_FLOP_PER_CLK_SM = 16384          # 8192 E4M3 multiply-adds per clock per SM
+FP8_SPEC_TFLOPS = 4500.0             # dense FP8, B200 specification
+HBM_SPEC_GBS = 8000.0
+
+
+def gemm_roofline(gemm_tflops: float, clocks: dict, peaks: dict) -> dict:
+    """The GEMM's rate against the FP8 peak that fits how it was timed.
+
+    The FP8 peak is the measured BF16 cuBLAS peak x 2 (nominal FP8 : BF16).
+    A short timed region that held the maximum SM clock with no power-cap
+    event compares with the burst figure; a region that ran under the power
+    cap (or whose clock was not sampled) with the sustained one."""
+    mhz, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    capped = "sw_power_cap" in clocks.get("reasons", [])
+    burst = mhz is not None and mx is not None and mhz >= 0.97 * mx and not capped
+    peak = 2.0 * (peaks["bf16"] if burst else peaks["bf16_sustained"])
+    alt = 2.0 * (peaks["bf16_sustained"] if burst else peaks["bf16"])
+    out = {"bound": "tensor", "achieved": gemm_tflops, "peak": peak, "unit": "TFLOP/s",
+           "frac": gemm_tflops / peak,
+           "peak_source": (f"{peaks['source']} {'burst' if burst else 'sustained'} bf16 "
+                           f"{peaks['bf16'] if burst else peaks['bf16_sustained']} TFLOP/s x 2 "
+                           f"(FP8 : BF16 nominal 2 : 1), chosen because the sampled SM clock "
+                           + ("stayed at its maximum with no power-cap event"
+                              if burst else "fell below its maximum or a power-cap event was seen")),
+           "frac_other_peak": gemm_tflops / alt,
+           "frac_spec": gemm_tflops / FP8_SPEC_TFLOPS}
+    if mhz:
+        ceiling = SM_COUNT * FP8_FLOP_PER_CLK_SM * mhz * 1e6 / 1e12
+        out.update(clock_ceiling=ceiling, frac_clock_ceiling=gemm_tflops / ceiling)
+    return out
+
+
+def run_config(desc: dict, world: int, host_inputs) -> dict:
+    """The config object of the JSON line (both arms print the same one)."""
+    cfg = dict(desc)
+    in_bytes = sum(t.numel() * t.element_size() for t in host_inputs) if host_inputs else 0
+    cfg.update(parallelism=f"replicas x{world}",
+               l2="inputs larger than L2 (no flush)" if in_bytes > L2_BYTES
+               else "inputs smaller than L2")
+    return cfg
 
 
 # ---------------------------------------------------------------- ncu traffic
@@ -256,15 +308,16 @@ def describe(workload):
         T = wl["x"].shape[0]
         M = int(lay.counts.sum())
         desc = dict(workload="moe grouped fprop, 32 experts W_e[2048,7168], 16384 tokens "
-                    "top-8 Zipf(1.1): 1x128 quantize tokens, FP8 dispatch to 128-padded "
-                    "groups, 128x128 quantize weights, grouped GEMM, bf16 out"
+                    "top-8 Zipf(1.1): 1x128 quantize tokens straight into their 128-padded "
+                    "expert groups, 128x128 quantize weights, grouped GEMM, bf16 out"
                     + (", pow2 scales applied in the tensor cores (UE8M0 block scaling)" if tc else ""),
                     M=M, N=N, K=K, M_padded=lay.m_total, tokens=T)
         inputs = [wl["x"], wl["w"], topk]
-        # tokens read once (2 B) + codes written (1 B); dispatched codes read
-        # once per token (1 B) and written per padded row (1 B); weights 3 B
-        quant_bytes = (T * K * 3 + T * K // 32 + (T + lay.m_total) * K + lay.m_total * K // 32
-                       + G * N * K * 3)
+        # tokens read once (2 B) and quantized straight into their padded
+        # expert rows (1 B code + 4/128 B scale per row element); weights
+        # read (2 B) and written as codes (1 B)
+        quant_bytes = (T * K * 2 + lay.m_total * K + lay.m_total * K // 32
+                       + G * N * K * 3 + G * (N // 128) * (K // 128) * 4)
 
         def make(d):
             if tc:
@@ -372,7 +425,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="fprop",
+    ap.add_argument("--workload", default="moe",
                     choices=["fprop", "fprop_pow2_tc", "pr1", "dgrad", "wgrad", "wgrad_pow2",
                              "wgrad_pow2_tc", "wgrad_cached", "moe", "moe_pow2_tc"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -403,7 +456,10 @@ def main():
                 "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": 2.0 * M * N * K / (v * 1e12) * 1e3, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": dict(described[1], parallelism="reference arm: CPU oracle, rank 0"),
+                "config": run_config(described[1], args.gpus, described[4]),
+                "timing": "the oracle on a bounded sample of the step, extrapolated to a "
+                          "whole step (rank 0, host cores)",
+                "ms_per_step_extrapolated": True,
                 "cpu_baseline": dict({k: res[k] for k in ("unit", "cores", "kind", "sample")},
                                      value=v),
                 "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -476,9 +532,7 @@ def main():
     ms_per_step = ms_total / args.steps
     value = job_throughput(world, flops, ms_per_step)
     peaks = measured_peaks()
-    # The GEMM is timed inside a long run of back-to-back steps: compare it
-    # with the sustained (power-capped) BF16 peak x 2 (FP8 : BF16 = 2 : 1).
-    fp8_peak = 2.0 * peaks["bf16_sustained"]
+    clock_summary = clocks.summary()
     gemm_tflops = flops / (gemm_avg * 1e-3) / 1e12
     quant_gbs = quant_bytes / (quant_avg * 1e-3) / 1e9
 
@@ -523,29 +577,30 @@ def main():
         cpu = {k: res[k] for k in ("value", "unit", "cores", "kind", "sample")}
 
     if rank == 0:
-        cfg = dict(desc)
-        cfg.update(parallelism=f"replicas x{world}", l2="inputs larger than L2 "
-                   "(no flush)" if sum(t.numel() * t.element_size() for t in host_inputs) > L2_BYTES
-                   else "inputs smaller than L2")
+        cfg = run_config(desc, world, host_inputs)
+        roof = gemm_roofline(gemm_tflops, clock_summary, peaks)
+        traffic = profiled_traffic(args.workload)
+        roof.update(traffic=traffic, kernel=gemm_kernel(args.workload),
+                    traffic_source=("ncu dram__bytes_read.sum + dram__bytes_write.sum of one "
+                                    "launch of the same kernel source on this workload, from "
+                                    f"profiles/{gemm_kernel(args.workload)}_{args.workload}.md"
+                                    if traffic is not None else
+                                    "no ncu capture of the current kernel source"))
         line = {
             "metric": "FP8 block-scaled GEMM TFLOP/s (step incl. quantization)",
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 x e4m3 -> f32",
             "data": "synthetic (seeded torch.Generator draws)", "config": cfg,
-            "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak,
-                         "unit": "TFLOP/s", "frac": gemm_tflops / fp8_peak,
-                         "traffic": profiled_traffic(args.workload),
-                         "kernel": gemm_kernel(args.workload), "peak_source":
-                         f"{peaks['source']} sustained bf16 {peaks['bf16_sustained']} TFLOP/s x 2 "
-                         f"(FP8/BF16 nominal); burst-based peak {2 * peaks['bf16']}"},
+            "roofline": roof,
             "quantizers": {"achieved_gbs": quant_gbs, "peak_gbs": peaks["hbm"],
-                           "frac": quant_gbs / peaks["hbm"], "ms_per_step": quant_avg,
+                           "frac": quant_gbs / peaks["hbm"],
+                           "frac_spec": quant_gbs / HBM_SPEC_GBS, "ms_per_step": quant_avg,
                            "algorithmic_bytes": quant_bytes},
             "gemm_ms": gemm_avg, "gemm_ms_min": gemm_ms[0],
             "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": step.kernel_calls * args.steps,
-            "clocks": clocks.summary(),
+            "clocks": clock_summary,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
