@@ -46,7 +46,7 @@ EXPORTED = (
     "fp8_set_wait_timeout_ns", "fp8_selftest_wait_timeout", "fp8_device_supported",
     "fp8_moe_dispatch_workspace_bytes", "fp8_moe_dispatch", "fp8_moe_combine",
     "fp8_moe_dispatch_noalloc", "fp8_requant_1x128_to_128x1", "fp8_blockscaled_gemm_pow2",
-    "fp8_grouped_gemm_pow2",
+    "fp8_grouped_gemm_pow2", "fp8_moe_quant_dispatch", "fp8_selftest_gemm_unwind",
 )
 
 
@@ -92,6 +92,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fp8_set_wait_timeout_ns.restype = None
     lib.fp8_selftest_wait_timeout.argtypes = [_P]
     lib.fp8_selftest_wait_timeout.restype = _I
+    lib.fp8_selftest_gemm_unwind.argtypes = [_I, _P, _P, _P, _P, _P, _I, _I64, _I64, _I64, _P,
+                                             _I, _P]
+    lib.fp8_selftest_gemm_unwind.restype = _I
     lib.fp8_device_supported.argtypes = []
     lib.fp8_device_supported.restype = _I
     lib.fp8_moe_dispatch_workspace_bytes.argtypes = [_I64, _I, _I]
@@ -101,6 +104,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fp8_moe_dispatch.restype = _I
     lib.fp8_moe_combine.argtypes = [_P, _I, _I64, _I64, _P, _P, _I64, _I, _P, _P]
     lib.fp8_moe_combine.restype = _I
+    lib.fp8_moe_quant_dispatch.argtypes = [_P, _I, _I64, _I64, _I64, _P, _I, _I, _P, _P, _I64,
+                                           _P, _P, _P, _P, _I64, _I, _P]
+    lib.fp8_moe_quant_dispatch.restype = _I
     lib.fp8_moe_dispatch_noalloc.argtypes = [_P, _P, _I64, _I64, _P, _I, _I, _P, _P, _I64, _P,
                                              _P, _P, _P]
     lib.fp8_moe_dispatch_noalloc.restype = _I
@@ -244,6 +250,21 @@ def fp8_moe_dispatch(q, sA, topk, G, q_out, sA_out, group_offsets, token_row, ro
         workspace.numel() * workspace.element_size(), _stream(stream)), "fp8_moe_dispatch")
 
 
+def fp8_moe_quant_dispatch(x, topk, G, q_out, sA_out, group_offsets, token_row, row_token,
+                           workspace, scale_mode: int = SCALE_FP32, stream=None) -> None:
+    """Tokens x [T,K] (BF16 or FP32) quantized 1x128 straight into the
+    expert-contiguous, 128-padded rows q_out [M_cap,K], sA_out [K/128,M_cap];
+    topk [T,k] int32."""
+    T, K = x.shape
+    k = topk.shape[1]
+    M_cap = q_out.shape[0]
+    _check(load_library().fp8_moe_quant_dispatch(
+        _ptr(x), _in_dtype(x), T, K, _row_stride(x), _ptr(topk), k, G, _ptr(q_out),
+        _ptr(sA_out), M_cap, _ptr(group_offsets), _ptr(token_row), _ptr(row_token),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), scale_mode,
+        _stream(stream)), "fp8_moe_quant_dispatch")
+
+
 def fp8_moe_dispatch_noalloc(q, sA, topk, G, q_out, sA_out, group_offsets, token_row, row_token,
                              stream=None) -> None:
     """fp8_moe_dispatch with the library's fixed device scratch (no workspace
@@ -277,6 +298,19 @@ def fp8_set_wait_timeout_ns(ns: int) -> None:
 
 def fp8_selftest_wait_timeout(stream=None) -> None:
     _check(load_library().fp8_selftest_wait_timeout(_stream(stream)), "fp8_selftest_wait_timeout")
+
+
+def fp8_selftest_gemm_unwind(kernel: int, A, sA, B, sB, D, group_offsets=None,
+                             stream=None) -> None:
+    """Launch GEMM `kernel` (0: software promotion, 1: tensor-core scaling) with
+    the odd CTA of every pair withholding its loads, so that its waits run out
+    (B [N,K] dense or [G,N,K] grouped)."""
+    M, K = A.shape
+    N = B.shape[-2]
+    G = B.shape[0] if group_offsets is not None else 0
+    _check(load_library().fp8_selftest_gemm_unwind(
+        kernel, _ptr(A), _ptr(sA), _ptr(B), _ptr(sB), _ptr(group_offsets), G, M, N, K, _ptr(D),
+        _out_dtype(D), _stream(stream)), "fp8_selftest_gemm_unwind")
 
 
 def fp8_device_supported() -> bool:

@@ -251,6 +251,39 @@ FP8FG_API int fp8_moe_dispatch(const uint8_t* q, const float* sA, int64_t T, int
                : FP8_ERR_LAUNCH;
 }
 
+FP8FG_API int fp8_moe_quant_dispatch(const void* x, int in_dtype, int64_t T, int64_t K,
+                                     int64_t ldx, const int32_t* topk, int k, int G,
+                                     uint8_t* q_out, float* sA_out, int64_t M_cap,
+                                     int32_t* group_offsets, int32_t* token_row,
+                                     int32_t* row_token, void* workspace, int64_t workspace_bytes,
+                                     int scale_mode, void* stream)
+{
+    if (!is_in(in_dtype) || !is_mode(scale_mode)) return FP8_ERR_DTYPE;
+    if (T < 0 || K <= 0 || K % 128 || K > kMaxDim || k < 1 || G < 1 || G > 1024 || M_cap < 0 ||
+        M_cap % 128 || M_cap > kMaxDim || T > kMaxPairs / k || (T + 127) / 128 > 65535 ||
+        ldx < K || ldx > kMaxDim)
+        return FP8_ERR_SHAPE;
+    if (workspace_bytes < fp8_moe_dispatch_workspace_bytes(T, k, G)) return FP8_ERR_SHAPE;
+    if (!group_offsets || (T > 0 && (!x || !topk || !token_row || !workspace)) ||
+        (M_cap > 0 && (!q_out || !sA_out || !row_token)))
+        return FP8_ERR_NULL;
+    if (!aligned(x, 16) || (ldx * in_size(in_dtype)) % 16 || !aligned(q_out, 16) ||
+        !aligned(sA_out, 4) || !aligned(topk, 4) || !aligned(group_offsets, 4) ||
+        !aligned(token_row, 4) || !aligned(row_token, 4) || !aligned(workspace, 4))
+        return FP8_ERR_ALIGN;
+    if (!device_is_sm100()) return FP8_ERR_DEVICE;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t* ws = static_cast<int32_t*>(workspace);
+    if (launch_moe_route(topk, T, k, G, M_cap, group_offsets, token_row, row_token, ws, st) !=
+            cudaSuccess ||
+        launch_quant_act_1x128_dispatch(x, in_dtype, T, K, ldx, token_row, k, M_cap, q_out,
+                                        sA_out, scale_mode, st) != cudaSuccess ||
+        launch_moe_rows(nullptr, nullptr, T, K, row_token, M_cap, q_out, sA_out, true, st) !=
+            cudaSuccess)
+        return FP8_ERR_LAUNCH;
+    return FP8_OK;
+}
+
 static_assert(kMoeStaticWsInts * (int64_t)sizeof(int32_t) == FP8_MOE_NOALLOC_WS_BYTES,
               "static dispatch scratch and its advertised size disagree");
 static int32_t g_no_device_ws = 0;
@@ -318,6 +351,30 @@ FP8FG_API int fp8_selftest_wait_timeout(void* stream)
     if (!device_is_sm100()) return FP8_ERR_DEVICE;
     return launch_selftest_wait(static_cast<cudaStream_t>(stream)) == cudaSuccess ? FP8_OK
                                                                                  : FP8_ERR_LAUNCH;
+}
+
+FP8FG_API int fp8_selftest_gemm_unwind(int kernel, const uint8_t* A, const float* sA,
+                                       const uint8_t* B, const float* sB,
+                                       const int32_t* group_offsets, int G, int64_t M, int64_t N,
+                                       int64_t K, void* D, int out_dtype, void* stream)
+{
+    if ((kernel != 0 && kernel != 1) || !is_out(out_dtype)) return FP8_ERR_DTYPE;
+    if (M <= 0 || M > kMaxDim || M % 128 || N <= 0 || N > kMaxDim || N % 128 || K < 256 ||
+        K > kMaxDim || K % 128 || (group_offsets && (G < 1 || G > 1024 || (int64_t)G * N > kMaxDim)))
+        return FP8_ERR_SHAPE;
+    if (!A || !sA || !B || !sB || !D) return FP8_ERR_NULL;
+    const int osz = out_dtype == FP8_OUT_BF16 ? 2 : 4;
+    if (!aligned(A, 16) || !aligned(B, 16) || !aligned(D, 16) || !aligned(sA, 4) ||
+        !aligned(sB, 4) || !aligned(group_offsets, 4) || (N * osz) % 16)
+        return FP8_ERR_ALIGN;
+    if (!device_is_sm100()) return FP8_ERR_DEVICE;
+    const int g = group_offsets ? G : 0;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return kernel == 0 ? launch_blockscaled_gemm_withheld(A, sA, B, FP8_B_KMAJOR, sB, 128, M, N, K,
+                                                          group_offsets, g, D, out_dtype, N, st)
+                       : launch_blockscaled_gemm_mx_withheld(A, sA, B, FP8_B_KMAJOR, sB, 128, M,
+                                                             N, K, group_offsets, g, D, out_dtype,
+                                                             N, st);
 }
 
 FP8FG_API int fp8_device_supported(void) { return device_is_sm100() ? 1 : 0; }

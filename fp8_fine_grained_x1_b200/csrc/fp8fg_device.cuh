@@ -1,9 +1,9 @@
 // fp8fg_device.cuh -- device-side building blocks of libfp8fg (sm_100a only).
 //
 // Inline-PTX wrappers for the Blackwell pieces the kernels are built from:
-// mbarriers, TMA tensor loads (no cluster multicast anywhere), tcgen05 MMA /
-// TMEM allocation / TMEM loads, packed FP32x2 FMA, and the library's status
-// word.  Every wait on an mbarrier is bounded: after a time limit it records
+// mbarriers, TMA tensor loads for CTA pairs (no cluster multicast
+// anywhere), tcgen05 MMA / TMEM allocation / TMEM loads, packed FP32x2 FMA,
+// and the library's status word.  Every wait on an mbarrier is bounded: after a time limit it records
 // FP8_ERR_TIMEOUT in the status word and reports failure to the caller, who
 // then unwinds (drains its own in-flight copies, frees TMEM, returns).
 #pragma once
@@ -179,64 +179,41 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// 2-D tiled tensor load global -> shared, completion counted in bytes on `bar`.
-// x is the innermost (contiguous) coordinate in elements.
-__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
-                                            int32_t x, int32_t y)
+// 2-D tiled tensor store shared -> global of the box at (x, y), tracked by
+// this thread's bulk async-group (x innermost, in elements; the parts of the
+// box outside the tensor are not written).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int32_t x,
+                                             int32_t y)
 {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-        : "memory");
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(smem_u32(smem_src))
+                 : "memory");
 }
 
-// Untiled bulk copy global -> shared (both 16-byte aligned, size % 16 == 0).
-__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes,
-                                          uint64_t* bar)
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Wait until at most N of this thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read()
 {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-            "r"(smem_u32(smem_dst)),
-        "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+// Wait until every bulk group of this thread has completed (writes done).
+__device__ __forceinline__ void bulk_wait_group_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (TMA stores, tcgen05 reads) before another thread starts one.
+__device__ __forceinline__ void fence_proxy_async_shared()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- tcgen05
 
-__device__ __forceinline__ void tmem_alloc(uint32_t* smem_dst, uint32_t ncols)
-{
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(smem_dst)),
-                 "r"(ncols)
-                 : "memory");
-}
-
-__device__ __forceinline__ void tmem_relinquish()
-{
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
-{
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-                 : "memory");
-}
-
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// D[tmem] (+)= A[smem] * B[smem], E4M3 x E4M3 -> FP32, one CTA.
-__device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                           uint32_t idesc, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
 
 // ---------------------------------------------------------------- CTA pairs
 // (2-CTA clusters: one tcgen05.mma.cta_group::2 spans the tensor cores of
@@ -327,14 +304,6 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t cta_mask
         " [%0], %1;" ::"r"(smem_u32(bar)),
         "h"(cta_mask)
         : "memory");
-}
-
-// Arrive (once) on `bar` when every tcgen05 op this thread issued has completed.
-__device__ __forceinline__ void mma_commit(uint64_t* bar)
-{
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     smem_u32(bar))
-                 : "memory");
 }
 
 // 32 consecutive FP32 columns of this thread's TMEM lane.
@@ -439,8 +408,8 @@ __device__ __forceinline__ void gemm_tile_coord(int64_t tile, int64_t nmb, int64
     mb = mb0 + r % rows;
 }
 
-// Group of the 128-row block starting at row0: the largest e with
-// off[e] <= row0; -1 when row0 >= off[G] (rows outside every group).
+// Group holding block index `row0` of a non-decreasing offset table: the
+// largest e with off[e] <= row0; -1 when row0 >= off[G].
 __device__ __forceinline__ int find_group(const int32_t* off, int G, int64_t row0)
 {
     int lo = 0, hi = G;
@@ -454,35 +423,33 @@ __device__ __forceinline__ int find_group(const int32_t* off, int G, int64_t row
     return lo < G ? lo : -1;
 }
 
-// The 128 rows of A (and of D) one CTA works on in m-block mb.
-//   dense            m0 = mb * tile_m + rank * 128, rows below M valid.
-//   grouped, single  m0 = mb * 128, in the group holding that row; blocks at
-//                    or past off[G] hold no group and are skipped (false).
-//   grouped, pairs   mb counts 256-row blocks group by group (poff), so a
-//                    pair never mixes two groups' rows (it shares one B); in
-//                    a group whose row count is an odd multiple of 128 the
-//                    last pair's odd CTA lies past the group end and idles.
+// The 128 rows of A (and of D) one CTA of a pair works on in m-block mb.
+//   dense    m0 = mb * 256 + rank * 128, rows below M valid.
+//   grouped  mb counts 256-row blocks group by group (poff), so a pair never
+//            mixes two groups' rows (it shares one B); in a group whose row
+//            count is an odd multiple of 128 the last pair's odd CTA lies
+//            past the group end and idles.  Blocks at or past poff[G] hold
+//            no group (false).
 struct TileRows {
     int g;           // group (0 when dense)
     int64_t m0;      // first row of this CTA's 128
     int64_t m_end;   // rows m0 .. m_end-1 belong to the tile's group
 };
 
-template <bool PAIR>
 __device__ __forceinline__ bool tile_rows(const int32_t* group_offsets, const int32_t* off,
                                           const int32_t* poff, int G, int64_t M, int64_t mb,
                                           uint32_t rank, TileRows& t)
 {
     if (!group_offsets) {
         t.g = 0;
-        t.m0 = mb * (PAIR ? 256 : 128) + rank * 128;
+        t.m0 = mb * 256 + rank * 128;
         t.m_end = M;
         return true;
     }
-    const int g = PAIR ? find_group(poff, G, mb) : find_group(off, G, mb * 128);
+    const int g = find_group(poff, G, mb);
     if (g < 0) return false;
     t.g = g;
-    t.m0 = PAIR ? off[g] + (mb - poff[g]) * 256 + rank * 128 : mb * 128;
+    t.m0 = off[g] + (mb - poff[g]) * 256 + rank * 128;
     t.m_end = off[g + 1];
     return true;
 }
@@ -512,10 +479,11 @@ __device__ __forceinline__ void pair_block_offsets(const int32_t* off, int32_t* 
 }
 
 // Host: 2-D uint8 tensor map [outer][inner], rows `row_bytes` apart, boxes of
-// box_inner x box_outer bytes, 128-byte swizzle, zero fill out of bounds
-// (defined in gemm.cu; false when the driver's encoder is unavailable).
+// box_inner x box_outer bytes, 128-byte swizzle (or none, with swizzle128 =
+// false), zero fill out of bounds (defined in gemm.cu; false when the
+// driver's encoder is unavailable).
 bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128 = true);
 
 // ---------------------------------------------------------------- registers
 

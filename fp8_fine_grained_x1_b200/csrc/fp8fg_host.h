@@ -28,6 +28,17 @@ int launch_blockscaled_gemm(const uint8_t* A, const float* sA, const uint8_t* B,
                             const int32_t* group_offsets, int G, void* D, int out_dtype,
                             int64_t ldd, cudaStream_t st);
 
+// Self-test forms of the two GEMMs: the odd CTA of every pair withholds its
+// operand loads after its first K-block, so the pair's waits run out.
+int launch_blockscaled_gemm_withheld(const uint8_t* A, const float* sA, const uint8_t* B,
+                                     int b_major, const float* sB, int sb_gran, int64_t M,
+                                     int64_t N, int64_t K, const int32_t* group_offsets, int G,
+                                     void* D, int out_dtype, int64_t ldd, cudaStream_t st);
+int launch_blockscaled_gemm_mx_withheld(const uint8_t* A, const float* sA, const uint8_t* B,
+                                        int b_major, const float* sB, int sb_gran, int64_t M,
+                                        int64_t N, int64_t K, const int32_t* group_offsets, int G,
+                                        void* D, int out_dtype, int64_t ldd, cudaStream_t st);
+
 cudaError_t launch_selftest_wait(cudaStream_t st);
 
 // MoE dispatch / combine (moe.cu).
@@ -36,6 +47,19 @@ cudaError_t launch_moe_dispatch(const uint8_t* q, const float* sA, int64_t T, in
                                 const int32_t* topk, int k, int G, uint8_t* q_out, float* sA_out,
                                 int64_t M_cap, int32_t* offsets, int32_t* token_row,
                                 int32_t* row_token, int32_t* ws, cudaStream_t st);
+// The dispatch in two halves: routing (group offsets, token_row, row_token)
+// and the row copy (pad_only: fill only the rows no pair claimed).
+cudaError_t launch_moe_route(const int32_t* topk, int64_t T, int k, int G, int64_t M_cap,
+                             int32_t* offsets, int32_t* token_row, int32_t* row_token, int32_t* ws,
+                             cudaStream_t st);
+cudaError_t launch_moe_rows(const uint8_t* q, const float* sA, int64_t T, int64_t K,
+                            const int32_t* row_token, int64_t M_cap, uint8_t* q_out,
+                            float* sA_out, bool pad_only, cudaStream_t st);
+// 1x128 quantization written straight to the rows token_row gives each token.
+cudaError_t launch_quant_act_1x128_dispatch(const void* x, int in_dtype, int64_t T, int64_t K,
+                                            int64_t ldx, const int32_t* token_row, int k,
+                                            int64_t M_cap, uint8_t* q_out, float* sA_out, int mode,
+                                            cudaStream_t st);
 cudaError_t launch_moe_combine(const void* D, int d_dtype, int64_t M_cap, int64_t N,
                                const int32_t* token_row, const float* w, int64_t T, int k, void* out,
                                cudaStream_t st);

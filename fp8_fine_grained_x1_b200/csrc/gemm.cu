@@ -36,8 +36,7 @@
 // TMEM buffer on the even CTA's `tempty` barrier.  Grouped (MoE) GEMMs count
 // their 256-row blocks group by group, so that both halves of a pair use the
 // same expert's B; a group of an odd number of 128-row blocks leaves the odd
-// CTA of its last pair idle.  Single CTAs remain the fallback when the device
-// cannot co-schedule 2-CTA clusters.
+// CTA of its last pair idle.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -56,18 +55,11 @@ namespace {
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 128;
+constexpr int TILE_M = 256;                             // rows per pair tile
 constexpr uint32_t A_BYTES = BM * BK;                   // 16 KB per stage
-constexpr uint32_t RING_BYTES = 4 * (A_BYTES + BN * BK); // 192 KB of stages
-constexpr int MAX_NS = 6;
-// Per-CTA tiling: a single CTA loads all 256 columns of B per K-block (48 KB
-// stages, 4 of them); a CTA of a pair loads 128 (32 KB stages, 6 of them).
-template <bool PAIR>
-struct Tiling {
-    static constexpr int TILE_M = PAIR ? 256 : 128;      // rows per MMA tile
-    static constexpr uint32_t B_BYTES = PAIR ? 128 * BK : BN * BK;
-    static constexpr int NS = (int)(RING_BYTES / (A_BYTES + B_BYTES));
-};
-static_assert(Tiling<true>::NS <= MAX_NS && Tiling<false>::NS <= MAX_NS, "ring barriers");
+constexpr uint32_t B_BYTES = 128 * BK;                  // this CTA's 128 of B's columns
+constexpr int NS = 6;                                   // ring stages of 32 KB
+constexpr uint32_t RING_BYTES = NS * (A_BYTES + B_BYTES);   // 192 KB
 constexpr int NUM_PROMO_WARPS = 8;
 constexpr int FIRST_PROMO_WARP = 4;                     // warpgroups 1 and 2
 constexpr int NUM_THREADS = 128 + 32 * NUM_PROMO_WARPS; // 384 = 3 warpgroups
@@ -82,7 +74,10 @@ static_assert(128 * CTRL_REGS + 256 * PROMO_REGS <= NUM_THREADS * LAUNCH_REGS,
 constexpr int PROMO_CHUNK = 32;                        // TMEM columns per load round trip
 constexpr uint32_t TMEM_COLS = 2 * BN;                  // two FP32 partial buffers
 constexpr int MAX_GROUPS = 1024;
-constexpr int BAND = 16;                                // m-blocks per raster band
+// Raster bands (m-blocks per band): 16 for dense GEMMs; 8 for grouped ones,
+// whose bands otherwise span several experts' rows and weights at once.
+constexpr int BAND_DENSE = 16;
+constexpr int BAND_GROUPED = 8;
 constexpr uint32_t DYN_SMEM = 1024 + RING_BYTES;
 
 struct GemmParams {
@@ -93,16 +88,24 @@ struct GemmParams {
     int64_t M, N, K, ldd;
     int G;
     int b_major, sb_gran, out_dtype;
-    int b_box_rows;                // rows of a K-major B box (128 or 256; 128 for pairs)
+    int band;                      // m-blocks per raster band
+    int withhold;                  // self-test: the odd CTA stops loading after one K-block
     uint64_t timeout_ns;
 };
 
 
-struct __align__(16) Shared {
+// Epilogue staging: each promotion warp writes its 32 rows x 32 bytes of
+// output at a time into one of two 1 KB buffers, from which a TMA store
+// copies them to D (EPI_COLS_B bytes wide, 32 rows).
+constexpr int EPI_BYTES = 32;                           // bytes of a row per store
+constexpr int EPI_ROWS = 32;
+
+struct __align__(128) Shared {
+    uint8_t epi[NUM_PROMO_WARPS][2][EPI_ROWS * EPI_BYTES];   // first: 128-byte aligned
     float sbw[NUM_PROMO_WARPS][2][128];   // per-warp column scales (sb_gran == 1),
-                                          // read and written as float4: first, 16-B aligned
-    uint64_t full[MAX_NS];
-    uint64_t empty[MAX_NS];
+                                          // read and written as float4: 16-B aligned
+    uint64_t full[NS];
+    uint64_t empty[NS];
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t drain;
@@ -113,6 +116,8 @@ struct __align__(16) Shared {
     int32_t poff[MAX_GROUPS + 1];   // grouped pairs: first 256-row block of each group
 };
 static_assert(offsetof(Shared, sbw) % 16 == 0, "float4 accesses need 16-byte alignment");
+static_assert(offsetof(Shared, epi) % 128 == 0 && EPI_ROWS * EPI_BYTES % 128 == 0,
+              "TMA store sources stay 128-byte aligned");
 static_assert(sizeof(float) * 128 % 16 == 0, "per-warp scale rows stay 16-byte aligned");
 static_assert(offsetof(Shared, full) % 8 == 0, "mbarriers need 8-byte alignment");
 
@@ -124,51 +129,45 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 
 // ------------------------------------------------------------------ roles
 
-template <bool PAIR>
 __device__ __forceinline__ bool tile_rows(const GemmParams& p, const Shared& sh, int64_t mb,
                                           uint32_t rank, TileRows& t)
 {
-    return tile_rows<PAIR>(p.group_offsets, sh.off, sh.poff, p.G, p.M, mb, rank, t);
+    return tile_rows(p.group_offsets, sh.off, sh.poff, p.G, p.M, mb, rank, t);
 }
 
-// Tiles are dealt round-robin to CTAs, or to pairs: pair c is CTAs 2c, 2c+1.
-template <bool PAIR>
+// Tiles are dealt round-robin to pairs: pair c is CTAs 2c, 2c+1.
 __device__ __forceinline__ void unit_range(int64_t& first, int64_t& stride)
 {
-    first = PAIR ? (int64_t)(blockIdx.x >> 1) : (int64_t)blockIdx.x;
-    stride = PAIR ? (int64_t)(gridDim.x >> 1) : (int64_t)gridDim.x;
+    first = (int64_t)(blockIdx.x >> 1);
+    stride = (int64_t)(gridDim.x >> 1);
 }
 
-template <bool PAIR>
 __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const GemmParams& p,
                              uint8_t* smem, Shared& sh, int64_t nmb, int64_t nnb, int64_t nkb)
 {
-    using T = Tiling<PAIR>;
-    constexpr int NS = T::NS;
     volatile int* abort = &sh.abort;
-    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    const uint32_t rank = cluster_ctarank();
     int64_t it = 0;   // loads issued so far; stage it % NS, round it / NS
     bool ok = true;
     int64_t first, stride;
-    unit_range<PAIR>(first, stride);
+    unit_range(first, stride);
     for (int64_t tile = first; ok && tile < nmb * nnb; tile += stride) {
         int64_t mb, nb;
-        gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
+        gemm_tile_coord(tile, nmb, nnb, p.band, mb, nb);
         TileRows tr;
-        if (!tile_rows<PAIR>(p, sh, mb, rank, tr)) continue;
+        if (!tile_rows(p, sh, mb, rank, tr)) continue;
         // (an idle odd CTA still loads its rows: the pair's MMA counts them)
         const int64_t m0 = tr.m0;
         const int64_t n0 = nb * BN;
         const int g = tr.g;
-        const int64_t n_valid = (p.N - n0 < BN) ? (p.N - n0) : BN;
-        // Bytes one CTA's B load(s) land per K-block (a box counts in full,
-        // its out-of-range part zero-filled).  A CTA of a pair loads B's
-        // columns rank*128 .. rank*128+127 of the tile.
-        const uint32_t b_bytes = PAIR                        ? 128u * BK
-                                 : p.b_major == FP8_B_KMAJOR ? (uint32_t)p.b_box_rows * BK
-                                                             : (uint32_t)n_valid * BK;
+        // A CTA of a pair loads B's columns rank*128 .. rank*128+127 of the
+        // tile (a box counts in full, its out-of-range part zero-filled).
         const int32_t brow = (int32_t)((int64_t)g * p.N + n0 + rank * 128);
         for (int64_t kb = 0; kb < nkb; ++kb) {
+            if (p.withhold && rank == 1 && it == 1) {   // self-test only
+                ok = false;
+                break;
+            }
             const int s = (int)(it % NS);
             const uint32_t ph = (uint32_t)((it / NS) & 1);
             if (!mbar_wait(&sh.empty[s], ph ^ 1u, abort, p.timeout_ns)) {
@@ -177,37 +176,23 @@ __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, con
             }
             ++it;
             uint8_t* a_dst = smem + s * A_BYTES;
-            uint8_t* b_dst = smem + NS * A_BYTES + s * T::B_BYTES;
-            if (PAIR) {
-                // Both CTAs' loads complete on the even CTA's barrier, which
-                // expects the pair's bytes; the odd CTA only issues its loads.
-                const uint32_t bar = mapa_shared(smem_u32(&sh.full[s]), 0);
-                if (rank == 0) mbar_arrive_expect_tx(&sh.full[s], 2 * (A_BYTES + b_bytes));
-                tma_load_2d_pair(a_dst, tmA, bar, (int32_t)(kb * BK), (int32_t)m0);
-                if (p.b_major == FP8_B_KMAJOR)
-                    tma_load_2d_pair(b_dst, tmB, bar, (int32_t)(kb * BK), brow);
-                else
-                    tma_load_2d_pair(b_dst, tmB, bar, (int32_t)(n0 + rank * 128),
-                                     (int32_t)(kb * BK));
-            } else {
-                mbar_arrive_expect_tx(&sh.full[s], A_BYTES + b_bytes);
-                tma_load_2d(a_dst, tmA, &sh.full[s], (int32_t)(kb * BK), (int32_t)m0);
-                if (p.b_major == FP8_B_KMAJOR) {
-                    tma_load_2d(b_dst, tmB, &sh.full[s], (int32_t)(kb * BK), brow);
-                } else {
-                    tma_load_2d(b_dst, tmB, &sh.full[s], (int32_t)n0, (int32_t)(kb * BK));
-                    if (n_valid > 128)
-                        tma_load_2d(b_dst + 128 * BK, tmB, &sh.full[s], (int32_t)(n0 + 128),
-                                    (int32_t)(kb * BK));
-                }
-            }
+            uint8_t* b_dst = smem + NS * A_BYTES + s * B_BYTES;
+            // Both CTAs' loads complete on the even CTA's barrier, which
+            // expects the pair's bytes; the odd CTA only issues its loads.
+            const uint32_t bar = mapa_shared(smem_u32(&sh.full[s]), 0);
+            if (rank == 0) mbar_arrive_expect_tx(&sh.full[s], 2 * (A_BYTES + B_BYTES));
+            tma_load_2d_pair(a_dst, tmA, bar, (int32_t)(kb * BK), (int32_t)m0);
+            if (p.b_major == FP8_B_KMAJOR)
+                tma_load_2d_pair(b_dst, tmB, bar, (int32_t)(kb * BK), brow);
+            else
+                tma_load_2d_pair(b_dst, tmB, bar, (int32_t)(n0 + rank * 128), (int32_t)(kb * BK));
         }
     }
     // Every copy issued must land before the CTA may exit: stage s received
     // ceil((it - s) / NS) loads, the last one completing phase (count-1)&1.
     // A pair's loads all count on the even CTA's barriers, so it drains for
     // both (the odd CTA stays resident until the closing cluster barrier).
-    if (PAIR && rank != 0) return;
+    if (rank != 0) return;
 #pragma unroll
     for (int s = 0; s < NS; ++s) {
         const int64_t count = it > s ? (it - s + NS - 1) / NS : 0;
@@ -215,12 +200,9 @@ __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, con
     }
 }
 
-template <bool PAIR>
 __device__ void run_mma(const GemmParams& p, uint8_t* smem, Shared& sh, int64_t nmb, int64_t nnb,
                         int64_t nkb)
 {
-    using T = Tiling<PAIR>;
-    constexpr int NS = T::NS;
     volatile int* abort = &sh.abort;
     const uint32_t a_base = smem_u32(smem);
     const uint32_t b_base = a_base + NS * A_BYTES;
@@ -228,17 +210,14 @@ __device__ void run_mma(const GemmParams& p, uint8_t* smem, Shared& sh, int64_t 
     int64_t it = 0, kbg = 0;
     bool ok = true;
     int64_t first, stride;
-    unit_range<PAIR>(first, stride);
+    unit_range(first, stride);
     for (int64_t tile = first; ok && tile < nmb * nnb; tile += stride) {
         int64_t mb, nb;
-        gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
-        const int64_t n0 = nb * BN;
-        if (!PAIR && p.group_offsets && find_group(sh.off, p.G, mb * BM) < 0) continue;
-        const int64_t n_valid = (p.N - n0 < BN) ? (p.N - n0) : BN;
+        gemm_tile_coord(tile, nmb, nnb, p.band, mb, nb);
+        (void)mb;
+        (void)nb;
         // A pair's MMA always spans 256 columns (a B tail is zero-filled).
-        const uint32_t idesc = idesc_e4m3_f32((uint32_t)T::TILE_M,
-                                              PAIR ? (uint32_t)BN : (uint32_t)n_valid,
-                                              (uint32_t)p.b_major);
+        const uint32_t idesc = idesc_e4m3_f32((uint32_t)TILE_M, (uint32_t)BN, (uint32_t)p.b_major);
         for (int64_t kb = 0; kb < nkb; ++kb, ++it, ++kbg) {
             const int s = (int)(it % NS);
             const uint32_t ph = (uint32_t)((it / NS) & 1);
@@ -252,42 +231,30 @@ __device__ void run_mma(const GemmParams& p, uint8_t* smem, Shared& sh, int64_t 
             tc_fence_after();
             const uint32_t d = tmem + buf * BN;
             const uint32_t a_addr = a_base + s * A_BYTES;
-            const uint32_t b_addr = b_base + s * T::B_BYTES;
+            const uint32_t b_addr = b_base + s * B_BYTES;
 #pragma unroll
             for (int k = 0; k < BK / 32; ++k) {
                 const uint64_t adesc = smem_desc_sw128(a_addr + k * 32, 16, 1024);
                 const uint64_t bdesc = (p.b_major == FP8_B_KMAJOR)
                                            ? smem_desc_sw128(b_addr + k * 32, 16, 1024)
                                            : smem_desc_sw128(b_addr + k * 32 * 128, 128 * BK, 1024);
-                if (PAIR)
-                    mma_f8f6f4_pair(d, adesc, bdesc, idesc, k > 0 ? 1u : 0u);
-                else
-                    mma_f8f6f4(d, adesc, bdesc, idesc, k > 0 ? 1u : 0u);
+                mma_f8f6f4_pair(d, adesc, bdesc, idesc, k > 0 ? 1u : 0u);
             }
-            if (PAIR) {
-                // stage free and partial ready in both CTAs of the pair
-                mma_commit_pair(&sh.empty[s], 3);
-                mma_commit_pair(&sh.tfull[buf], 3);
-            } else {
-                mma_commit(&sh.empty[s]);     // stage free once these MMAs are done
-                mma_commit(&sh.tfull[buf]);   // partial of this K-block ready
-            }
+            // stage free and partial ready in both CTAs of the pair
+            mma_commit_pair(&sh.empty[s], 3);
+            mma_commit_pair(&sh.tfull[buf], 3);
         }
     }
     // Wait for every MMA this thread issued before TMEM is released.
-    if (PAIR)
-        mma_commit_pair(&sh.drain, 1);
-    else
-        mma_commit(&sh.drain);
+    mma_commit_pair(&sh.drain, 1);
     mbar_wait_drain(&sh.drain, 0, p.timeout_ns);
 }
 
-template <bool PAIR>
-__device__ void run_promotion(const GemmParams& p, Shared& sh, int nmb, int nnb, int nkb, int warp,
-                              int lane)
+__device__ void run_promotion(const CUtensorMap* tmD, const GemmParams& p, Shared& sh, int nmb,
+                              int nnb, int nkb, int warp, int lane)
 {
     volatile int* abort = &sh.abort;
-    const int rank = PAIR ? (int)cluster_ctarank() : 0;
+    const int rank = (int)cluster_ctarank();
     const int ew = warp - FIRST_PROMO_WARP;   // 0..7
     const int quad = warp & 3;            // TMEM lanes this warp may access
     const int half = ew >> 2;             // column half of the tile
@@ -298,12 +265,12 @@ __device__ void run_promotion(const GemmParams& p, Shared& sh, int nmb, int nnb,
     uint32_t kbg = 0;
 
     int64_t first, stride;
-    unit_range<PAIR>(first, stride);
+    unit_range(first, stride);
     for (int tile = (int)first; tile < nmb * nnb; tile += (int)stride) {
         int64_t mb64, nb64;
-        gemm_tile_coord(tile, nmb, nnb, BAND, mb64, nb64);
+        gemm_tile_coord(tile, nmb, nnb, p.band, mb64, nb64);
         TileRows tr;
-        if (!tile_rows<PAIR>(p, sh, mb64, (uint32_t)rank, tr)) continue;
+        if (!tile_rows(p, sh, mb64, (uint32_t)rank, tr)) continue;
         const int nb = (int)nb64;
         const int m0 = (int)tr.m0, n0 = nb * BN;
         const int g = tr.g;
@@ -418,12 +385,8 @@ __device__ void run_promotion(const GemmParams& p, Shared& sh, int nmb, int nnb,
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                if (PAIR)   // the even CTA's MMA waits for both CTAs' warps
-                    mbar_arrive_cluster(mapa_shared(smem_u32(&sh.tempty[buf]), 0));
-                else
-                    mbar_arrive(&sh.tempty[buf]);
-            }
+            // the even CTA's MMA waits for both CTAs' warps
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&sh.tempty[buf]), 0));
             if (p.sb_gran == 1) {
                 *reinterpret_cast<float4*>(&sh.sbw[ew][(kb + 1) & 1][lane * 4]) = sb4_next;
                 __syncwarp();
@@ -431,37 +394,56 @@ __device__ void run_promotion(const GemmParams& p, Shared& sh, int nmb, int nnb,
         }
         if (!ok) break;
 
-        // Epilogue: round the FP32 sums to the output type and store the row.
-        if (active && row_ok) {
-            if (p.out_dtype == FP8_OUT_BF16) {
-                __nv_bfloat16* drow =
-                    static_cast<__nv_bfloat16*>(p.D) + (int64_t)m * p.ldd + n0 + col0;
+        // Epilogue: round the FP32 sums to the output type and store them.
+        // Each lane writes its row's next 32 bytes into this warp's staging
+        // buffer; one lane hands the 32 x 32-byte box to a TMA store, which
+        // drops the rows beyond M and the columns beyond N.  Two buffers
+        // alternate, so a store's read of one overlaps the writes of the other.
+        if (active) {
+            const int esz = p.out_dtype == FP8_OUT_BF16 ? 2 : 4;
+            const int nch = 128 * esz / EPI_BYTES;                 // 8 (BF16) or 16 (FP32)
+            const int32_t y = m0 + quad * 32;
+            const int32_t x0 = (n0 + col0) * esz;
 #pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    uint4 v;
-                    v.x = pack_bf16x2(acc[8 * c + 0], acc[8 * c + 1]);
-                    v.y = pack_bf16x2(acc[8 * c + 2], acc[8 * c + 3]);
-                    v.z = pack_bf16x2(acc[8 * c + 4], acc[8 * c + 5]);
-                    v.w = pack_bf16x2(acc[8 * c + 6], acc[8 * c + 7]);
-                    *reinterpret_cast<uint4*>(drow + 8 * c) = v;
+            for (int ch = 0; ch < 16; ++ch) {
+                if (ch >= nch) break;
+                uint8_t* buf = sh.epi[ew][ch & 1];
+                if (lane == 0) bulk_wait_group_read<1>();   // the store that read `buf` is done
+                __syncwarp();
+                uint4 w0, w1;
+                if (esz == 2) {
+                    const int j = 16 * ch;
+                    w0 = make_uint4(pack_bf16x2(acc[j + 0], acc[j + 1]), pack_bf16x2(acc[j + 2], acc[j + 3]),
+                                    pack_bf16x2(acc[j + 4], acc[j + 5]), pack_bf16x2(acc[j + 6], acc[j + 7]));
+                    w1 = make_uint4(pack_bf16x2(acc[j + 8], acc[j + 9]), pack_bf16x2(acc[j + 10], acc[j + 11]),
+                                    pack_bf16x2(acc[j + 12], acc[j + 13]), pack_bf16x2(acc[j + 14], acc[j + 15]));
+                } else {
+                    const int j = 8 * ch;
+                    w0 = make_uint4(__float_as_uint(acc[j + 0]), __float_as_uint(acc[j + 1]),
+                                    __float_as_uint(acc[j + 2]), __float_as_uint(acc[j + 3]));
+                    w1 = make_uint4(__float_as_uint(acc[j + 4]), __float_as_uint(acc[j + 5]),
+                                    __float_as_uint(acc[j + 6]), __float_as_uint(acc[j + 7]));
                 }
-            } else {
-                float* drow = static_cast<float*>(p.D) + (int64_t)m * p.ldd + n0 + col0;
-#pragma unroll
-                for (int c = 0; c < 32; ++c)
-                    *reinterpret_cast<float4*>(drow + 4 * c) =
-                        make_float4(acc[4 * c], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]);
+                *reinterpret_cast<uint4*>(buf + lane * EPI_BYTES) = w0;
+                *reinterpret_cast<uint4*>(buf + lane * EPI_BYTES + 16) = w1;
+                fence_proxy_async_shared();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(tmD, buf, x0 + ch * EPI_BYTES, y);
+                    bulk_commit_group();
+                }
             }
         }
     }
+    // every store has written D before the CTA exits
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
 }
 
-template <bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_fp8_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               const GemmParams p)
+               const __grid_constant__ CUtensorMap tmD, const GemmParams p)
 {
-    using T = Tiling<PAIR>;
     extern __shared__ uint8_t smem_raw[];
     __shared__ Shared sh;
     // Operand tiles need 1024-byte alignment (128-byte swizzle atoms).  The
@@ -473,17 +455,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int lane = threadIdx.x & 31;
     const int64_t nnb = (p.N + BN - 1) / BN;
     const int64_t nkb = p.K / BK;
-    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    const uint32_t rank = cluster_ctarank();
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < T::NS; ++s) {
+        for (int s = 0; s < NS; ++s) {
             mbar_init(&sh.full[s], 1);
             mbar_init(&sh.empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sh.tfull[b], 1);
-            // a pair's TMEM buffer is released by the promotion warps of both CTAs
-            mbar_init(&sh.tempty[b], PAIR ? 2 * NUM_PROMO_WARPS : NUM_PROMO_WARPS);
+            // a TMEM buffer is released by the promotion warps of both CTAs
+            mbar_init(&sh.tempty[b], 2 * NUM_PROMO_WARPS);
         }
         mbar_init(&sh.drain, 1);
         sh.abort = 0;
@@ -491,25 +473,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         fence_barrier_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmD);
     }
     if (warp == 1) {
-        if (PAIR) {
-            tmem_alloc_pair(&sh.tmem_base, TMEM_COLS);
-            tmem_relinquish_pair();
-        } else {
-            tmem_alloc(&sh.tmem_base, TMEM_COLS);
-            tmem_relinquish();
-        }
+        tmem_alloc_pair(&sh.tmem_base, TMEM_COLS);
+        tmem_relinquish_pair();
     }
     if (p.group_offsets)
         for (int i = threadIdx.x; i <= p.G; i += NUM_THREADS) sh.off[i] = p.group_offsets[i];
     // Barrier inits and the TMEM address must be visible to the peer CTA
     // before any of its loads, commits or arrives target them.
     tc_fence_before();
-    if (PAIR)
-        cluster_sync();
-    else
-        __syncthreads();
+    cluster_sync();
     tc_fence_after();
     if (p.group_offsets && threadIdx.x == 0) {
         bool bad = sh.off[0] != 0 || (int64_t)sh.off[p.G] > p.M;
@@ -521,39 +496,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     }
     __syncthreads();
-    if (PAIR && p.group_offsets && !sh.bad && warp == 0)
-        pair_block_offsets(sh.off, sh.poff, p.G, lane);
+    if (p.group_offsets && !sh.bad && warp == 0) pair_block_offsets(sh.off, sh.poff, p.G, lane);
     __syncthreads();
-    const int64_t nmb = (PAIR && p.group_offsets) ? (int64_t)sh.poff[p.G]
-                                                  : (p.M + T::TILE_M - 1) / T::TILE_M;
+    const int64_t nmb = p.group_offsets ? (int64_t)sh.poff[p.G] : (p.M + TILE_M - 1) / TILE_M;
 
     if (warp < FIRST_PROMO_WARP) {
         regs_dec<CTRL_REGS>();
         if (!sh.bad) {
             if (warp == 0) {
-                if (lane == 0) run_producer<PAIR>(&tmA, &tmB, p, smem, sh, nmb, nnb, nkb);
+                if (lane == 0) run_producer(&tmA, &tmB, p, smem, sh, nmb, nnb, nkb);
                 __syncwarp();
             } else if (warp == 1 && rank == 0) {   // a pair's MMAs issue from the even CTA
-                if (lane == 0) run_mma<PAIR>(p, smem, sh, nmb, nnb, nkb);
+                if (lane == 0) run_mma(p, smem, sh, nmb, nnb, nkb);
                 __syncwarp();
             }
         }
     } else {
         regs_inc<PROMO_REGS>();
-        if (!sh.bad) run_promotion<PAIR>(p, sh, (int)nmb, (int)nnb, (int)nkb, warp, lane);
+        if (!sh.bad) run_promotion(&tmD, p, sh, (int)nmb, (int)nnb, (int)nkb, warp, lane);
     }
     tc_fence_before();
-    if (PAIR)
-        cluster_sync();
-    else
-        __syncthreads();
+    cluster_sync();
     tc_fence_after();
-    if (warp == 1) {
-        if (PAIR)
-            tmem_dealloc_pair(sh.tmem_base, TMEM_COLS);
-        else
-            tmem_dealloc(sh.tmem_base, TMEM_COLS);
-    }
+    if (warp == 1) tmem_dealloc_pair(sh.tmem_base, TMEM_COLS);
 }
 
 __global__ void k_selftest_wait(uint64_t timeout_ns)
@@ -588,9 +553,8 @@ cudaLaunchConfig_t pair_launch_config(unsigned clusters, cudaStream_t st, cudaLa
     return cfg;
 }
 
-// Once per device: opt both kernels into the large dynamic shared memory and
-// ask how many CTA pairs fit at once (the persistent grid of the pair kernel;
-// 0 means pairs are unavailable and dense GEMMs run on single CTAs).
+// Once per device: opt the kernel into the large dynamic shared memory and
+// ask how many CTA pairs fit at once (the persistent grid).
 struct GemmDeviceSetup {
     bool ok = false;
     int pair_clusters = 0;
@@ -607,20 +571,20 @@ GemmDeviceSetup gemm_device_setup()
     if (!tried[dev]) {
         tried[dev] = true;
         GemmDeviceSetup r;
-        r.ok = cudaFuncSetAttribute(k_fp8_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)DYN_SMEM) == cudaSuccess &&
-               cudaFuncSetAttribute(k_fp8_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        r.ok = cudaFuncSetAttribute(k_fp8_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)DYN_SMEM) == cudaSuccess;
         if (r.ok) {
             cudaLaunchAttribute attr[1];
             const cudaLaunchConfig_t cfg =
                 pair_launch_config((unsigned)device_sm_count(), nullptr, attr);
             int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, k_fp8_gemm<true>, &cfg) != cudaSuccess) {
+            if (cudaOccupancyMaxActiveClusters(&n, k_fp8_gemm, &cfg) != cudaSuccess) {
                 n = 0;
                 (void)cudaGetLastError();
             }
             r.pair_clusters = n;
+        } else {
+            (void)cudaGetLastError();
         }
         done[dev] = r;
     }
@@ -650,9 +614,10 @@ EncodeTiledFn encode_fn()
 }
 
 // 2-D uint8 tensor [outer][inner] with rows `row_bytes` apart; boxes of
-// box_inner x box_outer bytes, 128-byte swizzle, zero fill out of bounds.
+// box_inner x box_outer bytes, 128-byte swizzle (or none), zero fill out of
+// bounds.
 bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer)
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
@@ -661,30 +626,38 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer
     const cuuint32_t box[2] = {box_inner, box_outer};
     const cuuint32_t estr[2] = {1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int launch_blockscaled_gemm(const uint8_t* A, const float* sA, const uint8_t* B, int b_major,
-                            const float* sB, int sb_gran, int64_t M, int64_t N, int64_t K,
-                            const int32_t* group_offsets, int G, void* D, int out_dtype,
-                            int64_t ldd, cudaStream_t st)
+namespace {
+
+int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, int b_major, const float* sB,
+                int sb_gran, int64_t M, int64_t N, int64_t K, const int32_t* group_offsets, int G,
+                void* D, int out_dtype, int64_t ldd, int withhold, cudaStream_t st)
 {
     if (M == 0) return FP8_OK;
     const GemmDeviceSetup setup = gemm_device_setup();
     if (!setup.ok) return FP8_ERR_LAUNCH;
-    const bool pair = setup.pair_clusters > 0;
+    if (setup.pair_clusters < 1) return FP8_ERR_DEVICE;   // needs co-scheduled 2-CTA clusters
     CUtensorMap tmA, tmB;
-    const int b_box_rows = pair ? 128 : (N >= BN ? BN : (int)N);
     if (!make_map(&tmA, A, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, BM)) return FP8_ERR_LAUNCH;
     bool okB;
     if (b_major == FP8_B_KMAJOR) {
         const uint64_t rows = (uint64_t)N * (uint64_t)(group_offsets ? G : 1);
-        okB = make_map(&tmB, B, (uint64_t)K, rows, (uint64_t)K, BK, (uint32_t)b_box_rows);
+        okB = make_map(&tmB, B, (uint64_t)K, rows, (uint64_t)K, BK, 128);
     } else {
         okB = make_map(&tmB, B, (uint64_t)N, (uint64_t)K, (uint64_t)N, 128, BK);
     }
     if (!okB) return FP8_ERR_LAUNCH;
+    // D as bytes: rows of N * element-size bytes, `ldd` elements apart; the
+    // epilogue stores 32-byte x 32-row boxes
+    CUtensorMap tmD;
+    const uint64_t esz = out_dtype == FP8_OUT_BF16 ? 2 : 4;
+    if (!make_map(&tmD, D, (uint64_t)N * esz, (uint64_t)M, (uint64_t)ldd * esz, EPI_BYTES, EPI_ROWS,
+                  false))
+        return FP8_ERR_LAUNCH;
     GemmParams p;
     p.sA = sA;
     p.sB = sB;
@@ -698,23 +671,36 @@ int launch_blockscaled_gemm(const uint8_t* A, const float* sA, const uint8_t* B,
     p.b_major = b_major;
     p.sb_gran = sb_gran;
     p.out_dtype = out_dtype;
-    p.b_box_rows = b_box_rows;
+    p.withhold = withhold;
+    p.band = group_offsets ? BAND_GROUPED : BAND_DENSE;
     p.timeout_ns = wait_timeout_ns();
-    if (pair) {
-        // grouped: each group adds at most one partly idle 256-row block
-        const int64_t tiles = ((M + 255) / 256 + (group_offsets ? G : 0)) * ((N + BN - 1) / BN);
-        const int64_t clusters = tiles < setup.pair_clusters ? tiles : setup.pair_clusters;
-        cudaLaunchAttribute attr[1];
-        const cudaLaunchConfig_t cfg = pair_launch_config((unsigned)clusters, st, attr);
-        return cudaLaunchKernelEx(&cfg, k_fp8_gemm<true>, tmA, tmB, p) == cudaSuccess
-                   ? FP8_OK
-                   : FP8_ERR_LAUNCH;
-    }
-    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
-    const int sms = device_sm_count();
-    const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
-    k_fp8_gemm<false><<<grid, NUM_THREADS, DYN_SMEM, st>>>(tmA, tmB, p);
-    return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_LAUNCH;
+    // grouped: each group adds at most one partly idle 256-row block
+    const int64_t tiles = ((M + 255) / 256 + (group_offsets ? G : 0)) * ((N + BN - 1) / BN);
+    const int64_t clusters = tiles < setup.pair_clusters ? tiles : setup.pair_clusters;
+    cudaLaunchAttribute attr[1];
+    const cudaLaunchConfig_t cfg = pair_launch_config((unsigned)clusters, st, attr);
+    return cudaLaunchKernelEx(&cfg, k_fp8_gemm, tmA, tmB, tmD, p) == cudaSuccess ? FP8_OK
+                                                                                  : FP8_ERR_LAUNCH;
+}
+
+}  // namespace
+
+int launch_blockscaled_gemm(const uint8_t* A, const float* sA, const uint8_t* B, int b_major,
+                            const float* sB, int sb_gran, int64_t M, int64_t N, int64_t K,
+                            const int32_t* group_offsets, int G, void* D, int out_dtype,
+                            int64_t ldd, cudaStream_t st)
+{
+    return launch_gemm(A, sA, B, b_major, sB, sb_gran, M, N, K, group_offsets, G, D, out_dtype,
+                       ldd, 0, st);
+}
+
+int launch_blockscaled_gemm_withheld(const uint8_t* A, const float* sA, const uint8_t* B,
+                                     int b_major, const float* sB, int sb_gran, int64_t M,
+                                     int64_t N, int64_t K, const int32_t* group_offsets, int G,
+                                     void* D, int out_dtype, int64_t ldd, cudaStream_t st)
+{
+    return launch_gemm(A, sA, B, b_major, sB, sb_gran, M, N, K, group_offsets, G, D, out_dtype,
+                       ldd, 1, st);
 }
 
 cudaError_t launch_selftest_wait(cudaStream_t st)

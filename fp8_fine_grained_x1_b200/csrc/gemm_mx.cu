@@ -82,18 +82,11 @@ constexpr int SF_AHEAD = 4;                 // K-blocks of scales each writer lo
 constexpr uint32_t SFA_BYTES = 512;              // 128 rows x 4 bytes
 constexpr uint32_t SFB_BYTES = 1024;             // 256 columns x 4 bytes
 constexpr uint32_t SF_BYTES = SFA_BYTES + SFB_BYTES;
-constexpr int MAX_NS = 6;
-constexpr uint32_t RING_BYTES = MAX_NS * (A_BYTES + 128 * BK + SF_BYTES);   // 201 KB
-// Per-CTA tiling: a single CTA loads all 256 columns of B per K-block (4
-// stages); a CTA of a pair loads 128 (6 stages).
-template <bool PAIR>
-struct MxTiling {
-    static constexpr int TILE_M = PAIR ? 256 : 128;
-    static constexpr uint32_t B_BYTES = PAIR ? 128 * BK : BN * BK;
-    static constexpr int NS = (int)(RING_BYTES / (A_BYTES + B_BYTES + SF_BYTES));
-};
-static_assert(MxTiling<true>::NS <= MAX_NS && MxTiling<false>::NS <= MAX_NS, "ring barriers");
-static_assert(SF_COL0 + MAX_NS * SF_SLOT_COLS <= TMEM_COLS, "scale slots exceed the allocation");
+constexpr int NS = 6;                       // ring stages
+constexpr int TILE_M = 256;                 // rows per pair tile
+constexpr uint32_t B_BYTES = 128 * BK;      // this CTA's 128 of B's columns
+constexpr uint32_t RING_BYTES = NS * (A_BYTES + B_BYTES + SF_BYTES);   // 201 KB
+static_assert(SF_COL0 + NS * SF_SLOT_COLS <= TMEM_COLS, "scale slots exceed the allocation");
 constexpr uint32_t DYN_SMEM = 1024 + RING_BYTES;
 
 constexpr int MAX_GROUPS = 1024;
@@ -106,13 +99,13 @@ struct MxParams {
     int64_t M, N, K, ldd;
     int G;
     int b_major, sb_gran, out_dtype;
-    int b_box_rows;
+    int withhold;        // self-test: the odd CTA stops loading after one K-block
     uint64_t timeout_ns;
 };
 
 struct __align__(8) MxShared {
-    uint64_t full[MAX_NS];     // operands landed (TMA bytes) and scales stored (scale warps)
-    uint64_t empty[MAX_NS];
+    uint64_t full[NS];         // operands landed (TMA bytes) and scales stored (scale warps)
+    uint64_t empty[NS];
     uint64_t acc_full;
     uint64_t acc_empty;
     uint64_t drain;
@@ -125,23 +118,10 @@ struct __align__(8) MxShared {
 
 // -------------------------------------------------------------- PTX helpers
 
-// Block-scaled MMA: D[tmem] (+)= (A * SFA) x (B * SFB), E4M3 operands from
-// shared memory, UE8M0 scale factors from TMEM, one CTA.
-__device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                         uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
-                                         uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::
-            "r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-        : "memory");
-}
-
-// The same over a CTA pair (M = 256: rows 0-127 in the even CTA, issued by
-// it; each CTA's scale factors from its own TMEM).
+// Block-scaled MMA over a CTA pair: D[tmem] (+)= (A * SFA) x (B * SFB),
+// E4M3 operands from shared memory, UE8M0 scale factors from TMEM (M = 256:
+// rows 0-127 in the even CTA, which issues it; each CTA's scale factors from
+// its own TMEM).
 __device__ __forceinline__ void mma_mxf8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                               uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
                                               uint32_t accumulate)
@@ -168,21 +148,10 @@ __host__ __device__ constexpr uint32_t idesc_mx_e4m3(uint32_t M, uint32_t N, uin
 }
 
 // Copy 32 lines of 16 bytes (a 512-byte block at `saddr`, no swizzle) from
-// shared memory to TMEM: line l -> lane l of every lane quarter, four 32-bit
-// columns from `taddr`.  Issued by the MMA thread; executes in order with
-// the tcgen05.mma instructions it issues afterwards.
-__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint32_t saddr)
-{
-    // descriptor: start >> 4; leading offset 16 B (unused: one 16-byte column);
-    // stride 128 B between groups of 8 lines; version 1; no swizzle
-    const uint64_t desc = (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)(16 >> 4) << 16) |
-                          ((uint64_t)(128 >> 4) << 32) | ((uint64_t)1 << 46);
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc)
-                 : "memory");
-}
-
-// The same for a CTA pair, issued by the even CTA: each CTA's 512-byte
-// block at `saddr` goes to that CTA's TMEM at `taddr`.
+// shared memory to TMEM, for both CTAs of a pair (issued by the even CTA:
+// each CTA's block goes to that CTA's TMEM at `taddr`): line l -> lane l of
+// every lane quarter, four 32-bit columns from `taddr`.  Executes in order
+// with the tcgen05.mma instructions issued after it.
 __device__ __forceinline__ void tmem_cp_32x128b_x4_pair(uint32_t taddr, uint32_t saddr)
 {
     const uint64_t desc = (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)(16 >> 4) << 16) |
@@ -228,45 +197,40 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 
 // ------------------------------------------------------------------ roles
 
-template <bool PAIR>
 __device__ __forceinline__ bool mx_tile_rows(const MxParams& p, const MxShared& sh, int64_t mb,
                                              uint32_t rank, TileRows& t)
 {
-    return tile_rows<PAIR>(p.group_offsets, sh.off, sh.poff, p.G, p.M, mb, rank, t);
+    return tile_rows(p.group_offsets, sh.off, sh.poff, p.G, p.M, mb, rank, t);
 }
 
-// Tiles are dealt round-robin to CTAs, or to pairs: pair c is CTAs 2c, 2c+1.
-template <bool PAIR>
+// Tiles are dealt round-robin to pairs: pair c is CTAs 2c, 2c+1.
 __device__ __forceinline__ void mx_unit_range(int64_t& first, int64_t& stride)
 {
-    first = PAIR ? (int64_t)(blockIdx.x >> 1) : (int64_t)blockIdx.x;
-    stride = PAIR ? (int64_t)(gridDim.x >> 1) : (int64_t)gridDim.x;
+    first = (int64_t)(blockIdx.x >> 1);
+    stride = (int64_t)(gridDim.x >> 1);
 }
 
-template <bool PAIR>
 __device__ void mx_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const MxParams& p,
                             uint8_t* smem, MxShared& sh, int64_t nmb, int64_t nnb, int64_t nkb)
 {
-    using T = MxTiling<PAIR>;
-    constexpr int NS = T::NS;
     volatile int* abort = &sh.abort;
-    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    const uint32_t rank = cluster_ctarank();
     int64_t it = 0;
     bool ok = true;
     int64_t first, stride;
-    mx_unit_range<PAIR>(first, stride);
+    mx_unit_range(first, stride);
     for (int64_t tile = first; ok && tile < nmb * nnb; tile += stride) {
         int64_t mb, nb;
         gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
         TileRows tr;
-        if (!mx_tile_rows<PAIR>(p, sh, mb, rank, tr)) continue;
+        if (!mx_tile_rows(p, sh, mb, rank, tr)) continue;
         const int64_t m0 = tr.m0, n0 = nb * BN;   // an idle odd CTA still loads
-        const int64_t n_valid = (p.N - n0 < BN) ? (p.N - n0) : BN;
-        const uint32_t b_bytes = PAIR                        ? 128u * BK
-                                 : p.b_major == FP8_B_KMAJOR ? (uint32_t)p.b_box_rows * BK
-                                                             : (uint32_t)n_valid * BK;
         const int32_t brow = (int32_t)((int64_t)tr.g * p.N + n0 + rank * 128);
         for (int64_t kb = 0; kb < nkb; ++kb) {
+            if (p.withhold && rank == 1 && it == 1) {   // self-test only
+                ok = false;
+                break;
+            }
             const int s = (int)(it % NS);
             const uint32_t ph = (uint32_t)((it / NS) & 1);
             if (!mbar_wait(&sh.empty[s], ph ^ 1u, abort, p.timeout_ns)) {
@@ -275,34 +239,20 @@ __device__ void mx_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, cons
             }
             ++it;
             uint8_t* a_dst = smem + s * A_BYTES;
-            uint8_t* b_dst = smem + NS * A_BYTES + s * T::B_BYTES;
-            if (PAIR) {
-                // both CTAs' bytes count on the even CTA's barrier
-                const uint32_t bar = mapa_shared(smem_u32(&sh.full[s]), 0);
-                if (rank == 0) mbar_arrive_expect_tx(&sh.full[s], 2 * (A_BYTES + b_bytes));
-                tma_load_2d_pair(a_dst, tmA, bar, (int32_t)(kb * BK), (int32_t)m0);
-                if (p.b_major == FP8_B_KMAJOR)
-                    tma_load_2d_pair(b_dst, tmB, bar, (int32_t)(kb * BK), brow);
-                else
-                    tma_load_2d_pair(b_dst, tmB, bar, (int32_t)(n0 + rank * 128),
-                                     (int32_t)(kb * BK));
-            } else {
-                mbar_arrive_expect_tx(&sh.full[s], A_BYTES + b_bytes);
-                tma_load_2d(a_dst, tmA, &sh.full[s], (int32_t)(kb * BK), (int32_t)m0);
-                if (p.b_major == FP8_B_KMAJOR) {
-                    tma_load_2d(b_dst, tmB, &sh.full[s], (int32_t)(kb * BK), brow);
-                } else {
-                    tma_load_2d(b_dst, tmB, &sh.full[s], (int32_t)n0, (int32_t)(kb * BK));
-                    if (n_valid > 128)
-                        tma_load_2d(b_dst + 128 * BK, tmB, &sh.full[s], (int32_t)(n0 + 128),
-                                    (int32_t)(kb * BK));
-                }
-            }
+            uint8_t* b_dst = smem + NS * A_BYTES + s * B_BYTES;
+            // both CTAs' bytes count on the even CTA's barrier
+            const uint32_t bar = mapa_shared(smem_u32(&sh.full[s]), 0);
+            if (rank == 0) mbar_arrive_expect_tx(&sh.full[s], 2 * (A_BYTES + B_BYTES));
+            tma_load_2d_pair(a_dst, tmA, bar, (int32_t)(kb * BK), (int32_t)m0);
+            if (p.b_major == FP8_B_KMAJOR)
+                tma_load_2d_pair(b_dst, tmB, bar, (int32_t)(kb * BK), brow);
+            else
+                tma_load_2d_pair(b_dst, tmB, bar, (int32_t)(n0 + rank * 128), (int32_t)(kb * BK));
         }
     }
     // every copy issued lands before the CTA exits (a pair's all count on the
     // even CTA's barriers; the odd CTA stays until the closing cluster barrier)
-    if (PAIR && rank != 0) return;
+    if (rank != 0) return;
 #pragma unroll
     for (int s = 0; s < NS; ++s) {
         const int64_t count = it > s ? (it - s + NS - 1) / NS : 0;
@@ -316,33 +266,27 @@ __device__ void mx_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, cons
 // idle.  The loop therefore waits for the next stage before issuing the
 // current stage's last MMA, so the barrier latency hides behind the MMAs
 // still executing, and it spins rather than suspends on barriers.
-template <bool PAIR>
 __device__ void mx_mma(const MxParams& p, uint8_t* smem, MxShared& sh, int64_t nmb, int64_t nnb,
                        int64_t nkb)
 {
-    using T = MxTiling<PAIR>;
-    constexpr int NS = T::NS;
     volatile int* abort = &sh.abort;
     const uint32_t a_base = smem_u32(smem);
     const uint32_t b_base = a_base + NS * A_BYTES;
-    const uint32_t sf_base = b_base + NS * T::B_BYTES;
+    const uint32_t sf_base = b_base + NS * B_BYTES;
     const uint32_t tmem = sh.tmem_base;
     const int64_t ntiles = nmb * nnb;
     uint32_t it = 0;          // K-blocks consumed so far (stage it % NS, round it / NS)
     uint32_t tcount = 0;
     bool ok = true;
     int64_t first, stride;
-    mx_unit_range<PAIR>(first, stride);
+    mx_unit_range(first, stride);
     for (int64_t tile = first; ok && tile < ntiles; tile += stride) {
         int64_t mb, nb;
         gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
-        if (!PAIR && p.group_offsets && find_group(sh.off, p.G, mb * BM) < 0) continue;
         const int64_t n0 = nb * BN;
-        const int64_t n_valid = (p.N - n0 < BN) ? (p.N - n0) : BN;
+        (void)n0;
         // a pair's MMA always spans 256 columns (a B tail is zero-filled)
-        const uint32_t idesc = idesc_mx_e4m3((uint32_t)T::TILE_M,
-                                             PAIR ? (uint32_t)BN : (uint32_t)n_valid,
-                                             (uint32_t)p.b_major);
+        const uint32_t idesc = idesc_mx_e4m3((uint32_t)TILE_M, (uint32_t)BN, (uint32_t)p.b_major);
         // the epilogue has read the previous tile's accumulator
         ok = mbar_wait_spin(&sh.acc_empty, (tcount & 1u) ^ 1u, abort, p.timeout_ns) &&
              mbar_wait_spin(&sh.full[it % NS], (it / NS) & 1u, abort, p.timeout_ns);
@@ -351,18 +295,12 @@ __device__ void mx_mma(const MxParams& p, uint8_t* smem, MxShared& sh, int64_t n
             const uint32_t s = it % NS;
             tc_fence_after();
             const uint32_t a_addr = a_base + s * A_BYTES;
-            const uint32_t b_addr = b_base + s * T::B_BYTES;
+            const uint32_t b_addr = b_base + s * B_BYTES;
             const uint32_t sf_addr = sf_base + s * SF_BYTES;
             const uint32_t sfa = tmem + SF_COL0 + s * SF_SLOT_COLS;
-            if (PAIR) {
-                tmem_cp_32x128b_x4_pair(sfa, sf_addr);
-                tmem_cp_32x128b_x4_pair(sfa + SFB_OFF, sf_addr + SFA_BYTES);
-                tmem_cp_32x128b_x4_pair(sfa + SFB_OFF + 4, sf_addr + SFA_BYTES + 512);
-            } else {
-                tmem_cp_32x128b_x4(sfa, sf_addr);                               // SFA, rows 0-127
-                tmem_cp_32x128b_x4(sfa + SFB_OFF, sf_addr + SFA_BYTES);         // SFB, columns 0-127
-                tmem_cp_32x128b_x4(sfa + SFB_OFF + 4, sf_addr + SFA_BYTES + 512);   // columns 128-255
-            }
+            tmem_cp_32x128b_x4_pair(sfa, sf_addr);                            // SFA, rows 0-127
+            tmem_cp_32x128b_x4_pair(sfa + SFB_OFF, sf_addr + SFA_BYTES);      // SFB, columns 0-127
+            tmem_cp_32x128b_x4_pair(sfa + SFB_OFF + 4, sf_addr + SFA_BYTES + 512);   // 128-255
 #pragma unroll
             for (int k = 0; k < BK / 32; ++k) {
                 if (k == BK / 32 - 1 && kb + 1 < nkb) {
@@ -378,30 +316,18 @@ __device__ void mx_mma(const MxParams& p, uint8_t* smem, MxShared& sh, int64_t n
                                            ? smem_desc_sw128(b_addr + k * 32, 16, 1024)
                                            : smem_desc_sw128(b_addr + k * 32 * 128, 128 * BK, 1024);
                 const uint32_t acc = (kb | k) ? 1u : 0u;
-                if (PAIR)
-                    mma_mxf8_pair(tmem, adesc, bdesc, idesc, sfa, sfa + SFB_OFF, acc);
-                else
-                    mma_mxf8(tmem, adesc, bdesc, idesc, sfa, sfa + SFB_OFF, acc);
+                mma_mxf8_pair(tmem, adesc, bdesc, idesc, sfa, sfa + SFB_OFF, acc);
             }
             // stage and scale slot free once these are done (in both CTAs)
-            if (PAIR)
-                mma_commit_pair(&sh.empty[s], 3);
-            else
-                mma_commit(&sh.empty[s]);
+            mma_commit_pair(&sh.empty[s], 3);
             if (!ok) break;
         }
         if (!ok) break;
         // the tile's sum is complete
-        if (PAIR)
-            mma_commit_pair(&sh.acc_full, 3);
-        else
-            mma_commit(&sh.acc_full);
+        mma_commit_pair(&sh.acc_full, 3);
         ++tcount;
     }
-    if (PAIR)
-        mma_commit_pair(&sh.drain, 1);
-    else
-        mma_commit(&sh.drain);
+    mma_commit_pair(&sh.drain, 1);
     mbar_wait_drain(&sh.drain, 0, p.timeout_ns);
 }
 
@@ -439,28 +365,25 @@ __device__ __forceinline__ void load_sf(const MxParams& p, int g, int64_t m0, in
 // line i % 32, word i / 32.
 __device__ __forceinline__ uint32_t sf_offset(int i) { return 16u * (uint32_t)(i & 31) + 4u * (uint32_t)(i >> 5); }
 
-template <bool PAIR>
 __device__ void mx_scale_writer(const MxParams& p, uint8_t* smem, MxShared& sh, int64_t nmb,
                                 int64_t nnb, int64_t nkb, int warp, int lane)
 {
-    using T = MxTiling<PAIR>;
-    constexpr int NS = T::NS;
     volatile int* abort = &sh.abort;
-    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    const uint32_t rank = cluster_ctarank();
     const int t = (warp - FIRST_SF_WARP) * 32 + lane;          // 0..127
-    uint8_t* sf_base = smem + NS * (A_BYTES + T::B_BYTES);
+    uint8_t* sf_base = smem + NS * (A_BYTES + B_BYTES);
     const uint32_t off_a = sf_offset(t);
     const uint32_t off_b0 = SFA_BYTES + sf_offset(t);
     const uint32_t off_b1 = SFA_BYTES + 512 + sf_offset(t);
     int64_t it = 0;
     bool ok = true, bad = false;
     int64_t first, stride;
-    mx_unit_range<PAIR>(first, stride);
+    mx_unit_range(first, stride);
     for (int64_t tile = first; ok && tile < nmb * nnb; tile += stride) {
         int64_t mb, nb;
         gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
         TileRows tr;
-        if (!mx_tile_rows<PAIR>(p, sh, mb, rank, tr)) continue;
+        if (!mx_tile_rows(p, sh, mb, rank, tr)) continue;
         const int64_t n0 = nb * BN;
         // SF_AHEAD K-blocks of scale loads in flight per thread
         SfRegs ring[SF_AHEAD];
@@ -488,12 +411,8 @@ __device__ void mx_scale_writer(const MxParams& p, uint8_t* smem, MxShared& sh, 
                         *reinterpret_cast<uint32_t*>(sf + off_b1) = wb1;
                         fence_proxy_async_smem();
                         __syncwarp();
-                        if (lane == 0) {
-                            if (PAIR)   // the even CTA's MMA thread copies both CTAs' blocks
-                                mbar_arrive_cluster(mapa_shared(smem_u32(&sh.full[s]), 0));
-                            else
-                                mbar_arrive(&sh.full[s]);
-                        }
+                        // the even CTA's MMA thread copies both CTAs' blocks
+                        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&sh.full[s]), 0));
                     } else {
                         ok = false;
                     }
@@ -504,12 +423,11 @@ __device__ void mx_scale_writer(const MxParams& p, uint8_t* smem, MxShared& sh, 
     if (__any_sync(0xffffffffu, bad) && lane == 0) report_error(FP8_ERR_VALUE);
 }
 
-template <bool PAIR>
 __device__ void mx_epilogue(const MxParams& p, MxShared& sh, int64_t nmb, int64_t nnb, int warp,
                             int lane)
 {
     volatile int* abort = &sh.abort;
-    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    const uint32_t rank = cluster_ctarank();
     const int ew = warp - FIRST_EPI_WARP;       // 0..7
     const int q = warp & 3;
     const int col0 = (ew >> 2) * 128;
@@ -517,12 +435,12 @@ __device__ void mx_epilogue(const MxParams& p, MxShared& sh, int64_t nmb, int64_
     const uint32_t taddr0 = sh.tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)col0;
     uint32_t tcount = 0;
     int64_t first, stride;
-    mx_unit_range<PAIR>(first, stride);
+    mx_unit_range(first, stride);
     for (int64_t tile = first; tile < nmb * nnb; tile += stride) {
         int64_t mb, nb;
         gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
         TileRows tr;
-        if (!mx_tile_rows<PAIR>(p, sh, mb, rank, tr)) continue;
+        if (!mx_tile_rows(p, sh, mb, rank, tr)) continue;
         const uint32_t tph = tcount++ & 1u;
         const int64_t m = tr.m0 + row;
         const int64_t n0 = nb * BN + col0;
@@ -541,12 +459,8 @@ __device__ void mx_epilogue(const MxParams& p, MxShared& sh, int64_t nmb, int64_
             if (c == 3) {                        // accumulator no longer needed
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) {
-                    if (PAIR)   // the even CTA's MMA waits for both CTAs' epilogues
-                        mbar_arrive_cluster(mapa_shared(smem_u32(&sh.acc_empty), 0));
-                    else
-                        mbar_arrive(&sh.acc_empty);
-                }
+                // the even CTA's MMA waits for both CTAs' epilogues
+                if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&sh.acc_empty), 0));
             }
             if (!(active && row_ok)) continue;
             if (p.out_dtype == FP8_OUT_BF16) {
@@ -571,12 +485,10 @@ __device__ void mx_epilogue(const MxParams& p, MxShared& sh, int64_t nmb, int64_
     }
 }
 
-template <bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_fp8_gemm_mx(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const MxParams p)
 {
-    using T = MxTiling<PAIR>;
     extern __shared__ uint8_t smem_raw[];
     __shared__ MxShared sh;
     // same 1024-byte-aligned offset in both CTAs of a pair
@@ -587,16 +499,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int lane = threadIdx.x & 31;
     const int64_t nnb = (p.N + BN - 1) / BN;
     const int64_t nkb = p.K / BK;
-    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    const uint32_t rank = cluster_ctarank();
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < T::NS; ++s) {
+        for (int s = 0; s < NS; ++s) {
             // the TMA bytes' arrive plus every scale warp (of both CTAs of a pair)
-            mbar_init(&sh.full[s], 1 + (PAIR ? 2 : 1) * NUM_SF_WARPS);
+            mbar_init(&sh.full[s], 1 + 2 * NUM_SF_WARPS);
             mbar_init(&sh.empty[s], 1);
         }
         mbar_init(&sh.acc_full, 1);
-        mbar_init(&sh.acc_empty, (PAIR ? 2 : 1) * NUM_EPI_WARPS);
+        mbar_init(&sh.acc_empty, 2 * NUM_EPI_WARPS);
         mbar_init(&sh.drain, 1);
         sh.abort = 0;
         sh.bad = 0;
@@ -605,22 +517,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tma_prefetch_desc(&tmB);
     }
     if (warp == 2) {
-        if (PAIR) {
-            tmem_alloc_pair(&sh.tmem_base, TMEM_COLS);
-            tmem_relinquish_pair();
-        } else {
-            tmem_alloc(&sh.tmem_base, TMEM_COLS);
-            tmem_relinquish();
-        }
+        tmem_alloc_pair(&sh.tmem_base, TMEM_COLS);
+        tmem_relinquish_pair();
     }
     if (p.group_offsets)
         for (int i = threadIdx.x; i <= p.G; i += NUM_THREADS) sh.off[i] = p.group_offsets[i];
     // barrier inits and the TMEM address visible to the peer CTA before use
     tc_fence_before();
-    if (PAIR)
-        cluster_sync();
-    else
-        __syncthreads();
+    cluster_sync();
     tc_fence_after();
     if (threadIdx.x == 0) {
         bool bad = false;
@@ -632,37 +536,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         sh.bad = bad ? 1 : 0;
     }
     __syncthreads();
-    if (PAIR && p.group_offsets && !sh.bad && warp == 0)
+    if (p.group_offsets && !sh.bad && warp == 0)
         pair_block_offsets(sh.off, sh.poff, p.G, lane);
     __syncthreads();
-    const int64_t nmb = (PAIR && p.group_offsets) ? (int64_t)sh.poff[p.G]
-                                                  : (p.M + T::TILE_M - 1) / T::TILE_M;
+    const int64_t nmb = p.group_offsets ? (int64_t)sh.poff[p.G] : (p.M + TILE_M - 1) / TILE_M;
 
     if (sh.bad) {
         // malformed offsets: nothing is loaded, multiplied or written
     } else if (warp == 0) {
-        if (lane == 0) mx_producer<PAIR>(&tmA, &tmB, p, smem, sh, nmb, nnb, nkb);
+        if (lane == 0) mx_producer(&tmA, &tmB, p, smem, sh, nmb, nnb, nkb);
         __syncwarp();
     } else if (warp == 1) {
-        if (lane == 0 && rank == 0) mx_mma<PAIR>(p, smem, sh, nmb, nnb, nkb);
+        if (lane == 0 && rank == 0) mx_mma(p, smem, sh, nmb, nnb, nkb);
         __syncwarp();
     } else if (warp >= FIRST_SF_WARP && warp < FIRST_SF_WARP + NUM_SF_WARPS) {
-        mx_scale_writer<PAIR>(p, smem, sh, nmb, nnb, nkb, warp, lane);
+        mx_scale_writer(p, smem, sh, nmb, nnb, nkb, warp, lane);
     } else if (warp >= FIRST_EPI_WARP) {
-        mx_epilogue<PAIR>(p, sh, nmb, nnb, warp, lane);
+        mx_epilogue(p, sh, nmb, nnb, warp, lane);
     }
     tc_fence_before();
-    if (PAIR)
-        cluster_sync();
-    else
-        __syncthreads();
+    cluster_sync();
     tc_fence_after();
-    if (warp == 2) {
-        if (PAIR)
-            tmem_dealloc_pair(sh.tmem_base, TMEM_COLS);
-        else
-            tmem_dealloc(sh.tmem_base, TMEM_COLS);
-    }
+    if (warp == 2) tmem_dealloc_pair(sh.tmem_base, TMEM_COLS);
 }
 
 cudaLaunchConfig_t mx_pair_config(unsigned clusters, cudaStream_t st, cudaLaunchAttribute* attr)
@@ -681,8 +576,8 @@ cudaLaunchConfig_t mx_pair_config(unsigned clusters, cudaStream_t st, cudaLaunch
     return cfg;
 }
 
-// Once per device: shared-memory opt-in for both kernels and the number of
-// CTA pairs that fit at once (0: pairs unavailable, single CTAs are used).
+// Once per device: shared-memory opt-in and the number of CTA pairs that fit
+// at once (the persistent grid).
 struct MxDeviceSetup {
     bool ok = false;
     int pair_clusters = 0;
@@ -699,45 +594,39 @@ MxDeviceSetup mx_device_setup()
     if (!tried[dev]) {
         tried[dev] = true;
         MxDeviceSetup r;
-        r.ok = cudaFuncSetAttribute(k_fp8_gemm_mx<false>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)DYN_SMEM) == cudaSuccess &&
-               cudaFuncSetAttribute(k_fp8_gemm_mx<true>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+        r.ok = cudaFuncSetAttribute(k_fp8_gemm_mx, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)DYN_SMEM) == cudaSuccess;
         if (r.ok) {
             cudaLaunchAttribute attr[1];
             const cudaLaunchConfig_t cfg = mx_pair_config((unsigned)device_sm_count(), nullptr, attr);
             int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, k_fp8_gemm_mx<true>, &cfg) != cudaSuccess) {
+            if (cudaOccupancyMaxActiveClusters(&n, k_fp8_gemm_mx, &cfg) != cudaSuccess) {
                 n = 0;
                 (void)cudaGetLastError();
             }
             r.pair_clusters = n;
+        } else {
+            (void)cudaGetLastError();
         }
         done[dev] = r;
     }
     return done[dev];
 }
 
-}  // namespace
-
-int launch_blockscaled_gemm_mx(const uint8_t* A, const float* sA, const uint8_t* B, int b_major,
-                               const float* sB, int sb_gran, int64_t M, int64_t N, int64_t K,
-                               const int32_t* group_offsets, int G, void* D, int out_dtype,
-                               int64_t ldd, cudaStream_t st)
+int launch_mx(const uint8_t* A, const float* sA, const uint8_t* B, int b_major, const float* sB,
+              int sb_gran, int64_t M, int64_t N, int64_t K, const int32_t* group_offsets, int G,
+              void* D, int out_dtype, int64_t ldd, int withhold, cudaStream_t st)
 {
     if (M == 0) return FP8_OK;
     const MxDeviceSetup setup = mx_device_setup();
     if (!setup.ok) return FP8_ERR_LAUNCH;
-    const bool pair = setup.pair_clusters > 0;
+    if (setup.pair_clusters < 1) return FP8_ERR_DEVICE;   // needs co-scheduled 2-CTA clusters
     CUtensorMap tmA, tmB;
-    const int b_box_rows = pair ? 128 : (N >= BN ? BN : (int)N);
     if (!make_map(&tmA, A, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, BM)) return FP8_ERR_LAUNCH;
     bool okB;
     if (b_major == FP8_B_KMAJOR) {
         const uint64_t rows = (uint64_t)N * (uint64_t)(group_offsets ? G : 1);
-        okB = make_map(&tmB, B, (uint64_t)K, rows, (uint64_t)K, BK, (uint32_t)b_box_rows);
+        okB = make_map(&tmB, B, (uint64_t)K, rows, (uint64_t)K, BK, 128);
     } else {
         okB = make_map(&tmB, B, (uint64_t)N, (uint64_t)K, (uint64_t)N, 128, BK);
     }
@@ -756,25 +645,37 @@ int launch_blockscaled_gemm_mx(const uint8_t* A, const float* sA, const uint8_t*
     p.b_major = b_major;
     p.sb_gran = sb_gran;
     p.out_dtype = out_dtype;
-    p.b_box_rows = b_box_rows;
+    p.withhold = withhold;
     p.timeout_ns = wait_timeout_ns();
 
     const int64_t nnb = (N + BN - 1) / BN;
-    if (pair) {
-        // grouped: each group adds at most one partly idle 256-row block
-        const int64_t tiles = ((M + 255) / 256 + (group_offsets ? G : 0)) * nnb;
-        const int64_t clusters = tiles < setup.pair_clusters ? tiles : setup.pair_clusters;
-        cudaLaunchAttribute attr[1];
-        const cudaLaunchConfig_t cfg = mx_pair_config((unsigned)clusters, st, attr);
-        return cudaLaunchKernelEx(&cfg, k_fp8_gemm_mx<true>, tmA, tmB, p) == cudaSuccess
-                   ? FP8_OK
-                   : FP8_ERR_LAUNCH;
-    }
-    const int64_t tiles = ((M + BM - 1) / BM) * nnb;
-    const int sms = device_sm_count();
-    const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
-    k_fp8_gemm_mx<false><<<grid, NUM_THREADS, DYN_SMEM, st>>>(tmA, tmB, p);
-    return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_LAUNCH;
+    // grouped: each group adds at most one partly idle 256-row block
+    const int64_t tiles = ((M + 255) / 256 + (group_offsets ? G : 0)) * nnb;
+    const int64_t clusters = tiles < setup.pair_clusters ? tiles : setup.pair_clusters;
+    cudaLaunchAttribute attr[1];
+    const cudaLaunchConfig_t cfg = mx_pair_config((unsigned)clusters, st, attr);
+    return cudaLaunchKernelEx(&cfg, k_fp8_gemm_mx, tmA, tmB, p) == cudaSuccess ? FP8_OK
+                                                                               : FP8_ERR_LAUNCH;
+}
+
+}  // namespace
+
+int launch_blockscaled_gemm_mx(const uint8_t* A, const float* sA, const uint8_t* B, int b_major,
+                               const float* sB, int sb_gran, int64_t M, int64_t N, int64_t K,
+                               const int32_t* group_offsets, int G, void* D, int out_dtype,
+                               int64_t ldd, cudaStream_t st)
+{
+    return launch_mx(A, sA, B, b_major, sB, sb_gran, M, N, K, group_offsets, G, D, out_dtype, ldd,
+                     0, st);
+}
+
+int launch_blockscaled_gemm_mx_withheld(const uint8_t* A, const float* sA, const uint8_t* B,
+                                        int b_major, const float* sB, int sb_gran, int64_t M,
+                                        int64_t N, int64_t K, const int32_t* group_offsets, int G,
+                                        void* D, int out_dtype, int64_t ldd, cudaStream_t st)
+{
+    return launch_mx(A, sA, B, b_major, sB, sb_gran, M, N, K, group_offsets, G, D, out_dtype, ldd,
+                     1, st);
 }
 
 int read_and_clear_mx_status() { return read_and_clear_module_status(); }

@@ -20,6 +20,7 @@
 //                 padding) and its 1x128 scales (or 1 for padding)
 // Padding rows get codes 0 and scale 1: exactly what quantizing a zero row
 // gives, so the result equals quantizing the gathered BF16 rows.
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -36,9 +37,9 @@ namespace {
 constexpr int kPairsPerChunk = 1024;
 
 
-// Fixed dispatch scratch for the non-allocating entry point (one per device
-// context).  Every entry a dispatch reads is written earlier in the same
-// dispatch, so it never needs clearing.
+// Fixed dispatch scratch for the non-allocating entry point (one per device,
+// in every context the module is loaded in).  Every entry a dispatch reads is
+// written earlier in the same dispatch, so it never needs clearing.
 __device__ __align__(256) int32_t g_moe_static_ws[kMoeStaticWsInts];
 
 __global__ void __launch_bounds__(256) k_moe_count(const int32_t* __restrict__ topk, int64_t P,
@@ -58,23 +59,39 @@ __global__ void __launch_bounds__(256) k_moe_count(const int32_t* __restrict__ t
     for (int e = threadIdx.x; e < G; e += blockDim.x) ws[(int64_t)blockIdx.x * G + e] = hist[e];
 }
 
-// One CTA; thread e walks the chunks of expert e.  ws[c][e] becomes the first
-// destination row of expert e's pairs in chunk c.
+// One CTA of 1024 threads.  Each expert e gets `tpe` consecutive threads
+// (the largest power of two with tpe * G <= 1024); thread `sub` of the group
+// sums a run of chunks of expert e, the group scans those sums in shared
+// memory, and each thread then rewrites its chunks with running bases.  In
+// the end ws[c][e] is the first destination row of expert e's pairs in chunk
+// c: the expert's padded group offset plus the pairs of earlier chunks.
 __global__ void __launch_bounds__(1024) k_moe_scan(int32_t* __restrict__ ws, int nchunks, int G,
                                                    int64_t M_cap, int32_t* __restrict__ offsets)
 {
+    __shared__ int32_t part[1024];
     __shared__ int32_t padded[1024];
     __shared__ int32_t base[1025];
-    const int e = threadIdx.x;
-    int32_t total = 0;
-    if (e < G) {
-        for (int c = 0; c < nchunks; ++c) {
-            const int32_t v = ws[(int64_t)c * G + e];
-            ws[(int64_t)c * G + e] = total;
-            total += v;
-        }
-        padded[e] = (total + 127) / 128 * 128;
+    int tpe = 1;
+    while (tpe * 2 * G <= 1024) tpe *= 2;
+    const int e = threadIdx.x / tpe;
+    const int sub = threadIdx.x % tpe;
+    const bool mine = e < G;
+    const int per = (nchunks + tpe - 1) / tpe;
+    const int c0 = sub * per < nchunks ? sub * per : nchunks;
+    const int c1 = c0 + per < nchunks ? c0 + per : nchunks;
+    int32_t sum = 0;
+    if (mine)
+        for (int c = c0; c < c1; ++c) sum += ws[(int64_t)c * G + e];
+    part[threadIdx.x] = sum;
+    __syncthreads();
+    // inclusive scan inside each group of tpe threads (Hillis-Steele)
+    for (int d = 1; d < tpe; d <<= 1) {
+        const int32_t add = (sub >= d) ? part[threadIdx.x - d] : 0;
+        __syncthreads();
+        part[threadIdx.x] += add;
+        __syncthreads();
     }
+    if (mine && sub == tpe - 1) padded[e] = (part[threadIdx.x] + 127) / 128 * 128;
     __syncthreads();
     if (threadIdx.x == 0) {
         int64_t acc = 0;
@@ -87,25 +104,41 @@ __global__ void __launch_bounds__(1024) k_moe_scan(int32_t* __restrict__ ws, int
     }
     __syncthreads();
     for (int j = threadIdx.x; j <= G; j += blockDim.x) offsets[j] = base[j];
-    if (e < G)
-        for (int c = 0; c < nchunks; ++c) ws[(int64_t)c * G + e] += base[e];
+    if (mine) {
+        int32_t run = base[e] + part[threadIdx.x] - sum;   // pairs of expert e before chunk c0
+        for (int c = c0; c < c1; ++c) {
+            const int32_t v = ws[(int64_t)c * G + e];
+            ws[(int64_t)c * G + e] = run;
+            run += v;
+        }
+    }
 }
 
-// One warp per chunk walks its pairs in order, 32 at a time.
+// One warp per chunk walks its pairs in order, 32 at a time.  The chunk's
+// expert ids are all loaded before the walk, so the walk itself waits on
+// shared memory only.
 __global__ void __launch_bounds__(32) k_moe_rank(const int32_t* __restrict__ topk, int64_t P, int k,
                                                  int G, const int32_t* __restrict__ ws,
                                                  int64_t M_cap, int32_t* __restrict__ token_row,
                                                  int32_t* __restrict__ row_token)
 {
     extern __shared__ int32_t cursor[];
+    constexpr int kSteps = kPairsPerChunk / 32;
     const int lane = threadIdx.x;
+    const int64_t i0 = (int64_t)blockIdx.x * kPairsPerChunk;
+    int32_t ids[kSteps];
+#pragma unroll
+    for (int j = 0; j < kSteps; ++j) {
+        const int64_t idx = i0 + j * 32 + lane;
+        ids[j] = idx < P ? __ldg(topk + idx) : -1;
+    }
     for (int e = lane; e < G; e += 32) cursor[e] = ws[(int64_t)blockIdx.x * G + e];
     __syncwarp();
-    const int64_t i0 = (int64_t)blockIdx.x * kPairsPerChunk;
-    for (int s = 0; s < kPairsPerChunk; s += 32) {
-        const int64_t idx = i0 + s + lane;
+#pragma unroll
+    for (int j = 0; j < kSteps; ++j) {
+        const int64_t idx = i0 + j * 32 + lane;
         const bool live = idx < P;
-        int32_t e = live ? topk[idx] : -1;
+        int32_t e = ids[j];
         const bool ok = live && e >= 0 && e < G;
         if (live && !ok) report_error(FP8_ERR_SHAPE);
         if (!ok) e = -1 - lane;                 // unique key: never matches another lane
@@ -126,12 +159,14 @@ __global__ void __launch_bounds__(32) k_moe_rank(const int32_t* __restrict__ top
 }
 
 // CTA = 8 warps, one destination row per warp: the row's K code bytes in
-// 16-byte vectors, then its K/128 scales.
+// 16-byte vectors, then its K/128 scales.  With `pad_only` the rows that hold
+// a pair are left alone (their codes were written by the quantizer itself)
+// and only the padding rows are filled.
 __global__ void __launch_bounds__(256) k_moe_rows(const uint8_t* __restrict__ q,
                                                   const float* __restrict__ sA, int64_t T, int64_t K,
                                                   const int32_t* __restrict__ row_token,
                                                   int64_t M_cap, uint8_t* __restrict__ q_out,
-                                                  float* __restrict__ sA_out)
+                                                  float* __restrict__ sA_out, bool pad_only)
 {
     const int lane = threadIdx.x & 31;
     const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -140,6 +175,7 @@ __global__ void __launch_bounds__(256) k_moe_rows(const uint8_t* __restrict__ q,
     uint4* dst = reinterpret_cast<uint4*>(q_out + r * K);
     const int64_t nvec = K / 16;
     if (t >= 0 && t < T) {
+        if (pad_only) return;
         const uint4* src = reinterpret_cast<const uint4*>(q + (int64_t)t * K);
         for (int64_t v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
         for (int64_t kb = lane; kb < K / 128; kb += 32) sA_out[kb * M_cap + r] = __ldg(sA + kb * T + t);
@@ -202,10 +238,10 @@ int64_t moe_dispatch_workspace_ints(int64_t P, int G)
     return ((P + kPairsPerChunk - 1) / kPairsPerChunk) * (int64_t)G;
 }
 
-cudaError_t launch_moe_dispatch(const uint8_t* q, const float* sA, int64_t T, int64_t K,
-                                const int32_t* topk, int k, int G, uint8_t* q_out, float* sA_out,
-                                int64_t M_cap, int32_t* offsets, int32_t* token_row,
-                                int32_t* row_token, int32_t* ws, cudaStream_t st)
+// Routing half of the dispatch: group offsets, token_row and row_token.
+cudaError_t launch_moe_route(const int32_t* topk, int64_t T, int k, int G, int64_t M_cap,
+                             int32_t* offsets, int32_t* token_row, int32_t* row_token, int32_t* ws,
+                             cudaStream_t st)
 {
     const int64_t P = T * k;
     const int nchunks = (int)((P + kPairsPerChunk - 1) / kPairsPerChunk);
@@ -223,10 +259,29 @@ cudaError_t launch_moe_dispatch(const uint8_t* q, const float* sA, int64_t T, in
                                                             row_token);
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
     }
+    return cudaSuccess;
+}
+
+// Row half: copy each claimed row's codes and scales from the token's, and
+// fill the padding rows (or, with pad_only, fill the padding rows only).
+cudaError_t launch_moe_rows(const uint8_t* q, const float* sA, int64_t T, int64_t K,
+                            const int32_t* row_token, int64_t M_cap, uint8_t* q_out,
+                            float* sA_out, bool pad_only, cudaStream_t st)
+{
     if (M_cap > 0)
         k_moe_rows<<<(unsigned)((M_cap + 7) / 8), 256, 0, st>>>(q, sA, T, K, row_token, M_cap,
-                                                              q_out, sA_out);
+                                                              q_out, sA_out, pad_only);
     return cudaGetLastError();
+}
+
+cudaError_t launch_moe_dispatch(const uint8_t* q, const float* sA, int64_t T, int64_t K,
+                                const int32_t* topk, int k, int G, uint8_t* q_out, float* sA_out,
+                                int64_t M_cap, int32_t* offsets, int32_t* token_row,
+                                int32_t* row_token, int32_t* ws, cudaStream_t st)
+{
+    cudaError_t err = launch_moe_route(topk, T, k, G, M_cap, offsets, token_row, row_token, ws, st);
+    if (err != cudaSuccess) return err;
+    return launch_moe_rows(q, sA, T, K, row_token, M_cap, q_out, sA_out, false, st);
 }
 
 cudaError_t launch_moe_combine(const void* D, int d_dtype, int64_t M_cap, int64_t N,
@@ -245,21 +300,51 @@ cudaError_t launch_moe_combine(const void* D, int d_dtype, int64_t M_cap, int64_
     return cudaGetLastError();
 }
 
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// The driver's cuCtxGetCurrent, looked up once (the runtime is linked
+// statically; the driver is reached through its entry-point table).
+CtxGetCurrentFn ctx_get_current()
+{
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(f);
+    });
+    return fn;
+}
+
+// Device address of g_moe_static_ws in the current context.  A __device__
+// array has one address per context the module is loaded in, so the address
+// is cached per device together with the context it was looked up in, and
+// looked up again when the caller's current context is another one.
 cudaError_t moe_static_workspace(int32_t** ws)
 {
     constexpr int kMaxDevices = 64;
     static std::mutex mu;
     static int32_t* addr[kMaxDevices] = {};
+    static CUcontext ctx_of[kMaxDevices] = {};
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    const CtxGetCurrentFn get_ctx = ctx_get_current();
+    CUcontext ctx = nullptr;
+    if (get_ctx && get_ctx(&ctx) != CUDA_SUCCESS) ctx = nullptr;
     std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
+    if (!addr[dev] || ctx_of[dev] != ctx) {
         void* p = nullptr;
-        err = cudaGetSymbolAddress(&p, g_moe_static_ws);     // for the current device
+        err = cudaGetSymbolAddress(&p, g_moe_static_ws);     // with this device current
         if (err != cudaSuccess) return err;
         addr[dev] = static_cast<int32_t*>(p);
+        // the lookup makes the device's primary context current if no
+        // context was: remember the one current now
+        if (get_ctx && get_ctx(&ctx) != CUDA_SUCCESS) ctx = nullptr;
+        ctx_of[dev] = ctx;
     }
     *ws = addr[dev];
     return cudaSuccess;

@@ -187,6 +187,62 @@ __global__ void __launch_bounds__(256) k_quant_1x128(const Tin* __restrict__ x, 
     }
 }
 
+// 1x128 quantization straight into the MoE dispatch layout: the same groups,
+// scales and codes as k_quant_1x128, but each token's codes and scales are
+// written to every destination row its routing gave it (token_row[t][j],
+// j < k; -1 means the pair was dropped) instead of to the token's own row.
+// The token's codes never round-trip through HBM before the dispatch.
+// Lanes 0..k-1 of each half-warp fetch the token's destinations; a shuffle
+// hands them to the other lanes.  Grid and CTA as k_quant_1x128.
+template <typename Tin>
+__global__ void __launch_bounds__(256) k_quant_1x128_dispatch(
+    const Tin* __restrict__ x, int64_t T, int64_t ldx, const int32_t* __restrict__ token_row,
+    int k, int64_t M_cap, uint8_t* __restrict__ q_out, int64_t K, float* __restrict__ sA_out,
+    int mode)
+{
+    const int h = threadIdx.x >> 4;
+    const int l = threadIdx.x & 15;
+    const unsigned half_mask = 0xFFFFu << (threadIdx.x & 16);
+    const int64_t kb = blockIdx.x;
+    const int64_t t0 = (int64_t)blockIdx.y * kRowsPerCta1x128;
+
+    Chunk8<Tin> c[kGroupsPerThread1x128];
+#pragma unroll
+    for (int u = 0; u < kGroupsPerThread1x128; ++u) {
+        const int64_t t = t0 + u * 16 + h;
+        if (t < T)
+            c[u].load(x + t * ldx + kb * 128 + l * 8);
+        else
+            c[u].zero();
+    }
+#pragma unroll
+    for (int u = 0; u < kGroupsPerThread1x128; ++u) {
+        const int64_t t = t0 + u * 16 + h;
+        float v[8];
+        c[u].get(v);
+        float a = absmax8(v);
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 8));
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+        const GroupScale g = group_scale(a, mode);
+        uint2 out;
+        out.x = encode4(v[0], v[1], v[2], v[3], g.inv);
+        out.y = encode4(v[4], v[5], v[6], v[7], g.inv);
+        const bool live = t < T;
+        for (int j0 = 0; j0 < k; j0 += 16) {
+            const int32_t mine = (live && j0 + l < k) ? __ldg(token_row + t * k + j0 + l) : -1;
+            const int nj = k - j0 < 16 ? k - j0 : 16;
+            for (int j = 0; j < nj; ++j) {
+                const int32_t r = __shfl_sync(half_mask, mine, j, 16);
+                if (r < 0 || r >= M_cap) continue;
+                *reinterpret_cast<uint2*>(q_out + (int64_t)r * K + kb * 128 + l * 8) = out;
+                if (l == 0) sA_out[kb * M_cap + r] = g.s;
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------------ 128x128
 
 // CTA = 256 threads per 128x128 block: thread (r0 = tid/16, c = tid%16) loads
@@ -567,6 +623,24 @@ cudaError_t launch_quant_act_1x128(const void* x, int in_dtype, int64_t M, int64
     else
         k_quant_1x128<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), M, ldx, q, ldq,
                                                    sA, mode);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_act_1x128_dispatch(const void* x, int in_dtype, int64_t T, int64_t K,
+                                            int64_t ldx, const int32_t* token_row, int k,
+                                            int64_t M_cap, uint8_t* q_out, float* sA_out, int mode,
+                                            cudaStream_t st)
+{
+    if (T == 0) return cudaSuccess;
+    const dim3 grid((unsigned)(K / 128), (unsigned)((T + kRowsPerCta1x128 - 1) / kRowsPerCta1x128));
+    if (in_dtype == FP8_IN_BF16)
+        k_quant_1x128_dispatch<__nv_bfloat16><<<grid, 256, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(x), T, ldx, token_row, k, M_cap, q_out, K, sA_out,
+            mode);
+    else
+        k_quant_1x128_dispatch<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), T, ldx,
+                                                            token_row, k, M_cap, q_out, K, sA_out,
+                                                            mode);
     return cudaGetLastError();
 }
 

@@ -12,8 +12,9 @@ called, issues only library calls on the current stream:
                per-channel scales; dW[C_out,C_in] = dY^T . X, FP32 out
   WgradCachedStep  as WgradStep, with X taken from its cached 1x128 FP8
                form and requantized into 128x1 groups
-  MoeStep      tokens X[T,K] --1x128-->, FP8 dispatch of the rows to
-               expert-contiguous groups; W[G,N,K] --128x128-->; grouped GEMM
+  MoeStep      tokens X[T,K] --1x128, written straight to their expert-
+               contiguous, 128-padded FP8 rows-->; W[G,N,K] --128x128-->;
+               grouped GEMM
 
 ("5 Ways You can get More Deepseek While Spending Less", Figure 6: Fprop,
 Dgrad and Wgrad all run in FP8; why-be.co.kr / cameseeing.com posts and
@@ -33,7 +34,7 @@ import torch
 
 from . import (B_KMAJOR, B_MNMAJOR, SCALE_FP32, SCALE_POW2, fp8_blockscaled_gemm,
                fp8_blockscaled_gemm_pow2, fp8_grouped_gemm, fp8_grouped_gemm_pow2,
-               fp8_moe_combine, fp8_moe_dispatch, fp8_moe_dispatch_workspace_bytes,
+               fp8_moe_combine, fp8_moe_dispatch_workspace_bytes, fp8_moe_quant_dispatch,
                fp8_quant_act_128x1, fp8_quant_act_1x128, fp8_quant_w_128x128,
                fp8_requant_1x128_to_128x1, moe_capacity)
 
@@ -178,11 +179,13 @@ class WgradCachedStep:
 
 
 class MoeStep:
-    """MoE expert layer forward: tokens X[T,K] --1x128--> FP8 rows, FP8
-    dispatch to expert-contiguous 128-padded groups (fp8_moe_dispatch),
+    """MoE expert layer forward: tokens X[T,K] --1x128 quantized straight
+    into expert-contiguous, 128-padded FP8 groups (fp8_moe_quant_dispatch)-->,
     W[G,N,K] --128x128-->, grouped GEMM.  `combine(weights)` adds the
     weighted return to token order."""
-    kernel_calls = 7      # quantize X, 4 dispatch kernels, quantize W, grouped GEMM (+1 memset)
+    # routing (count, scan, rank), fused quantizer, padding rows, quantize W,
+    # grouped GEMM (+1 memset)
+    kernel_calls = 7
 
     def __init__(self, x, topk, w, out_dtype=torch.bfloat16, scale_mode=SCALE_FP32,
                  tensor_core_scaling=False):
@@ -195,8 +198,6 @@ class MoeStep:
         k = topk.shape[1]
         d = x.device
         self.x, self.topk, self.w, self.mode, self.G = x, topk, w, scale_mode, G
-        self.qx = _empty((T, K), torch.uint8, d)
-        self.sx = _empty((K // 128, T), torch.float32, d)
         self.M_cap = moe_capacity(T, k, G)
         self.qa = _empty((self.M_cap, K), torch.uint8, d)
         self.sa = _empty((K // 128, self.M_cap), torch.float32, d)
@@ -211,9 +212,8 @@ class MoeStep:
         self.inputs, self.output = [x, w, topk], self.y
 
     def quantize(self, stream=None):
-        fp8_quant_act_1x128(self.x, self.qx, self.sx, self.mode, stream)
-        fp8_moe_dispatch(self.qx, self.sx, self.topk, self.G, self.qa, self.sa, self.offsets,
-                         self.token_row, self.row_token, self.ws, stream)
+        fp8_moe_quant_dispatch(self.x, self.topk, self.G, self.qa, self.sa, self.offsets,
+                               self.token_row, self.row_token, self.ws, self.mode, stream)
         G, N, K = self.w.shape
         fp8_quant_w_128x128(self.w.view(G * N, K), self.qw.view(G * N, K),
                             self.sw.view(G * N // 128, K // 128), self.mode, stream)

@@ -30,6 +30,9 @@
  *     keeps no per-call state; its only global state is two status words per
  *     device (__device__ variables: one for the GEMM, one for the MoE
  *     dispatch) and a host-side wait time limit.
+ *   - Per-device set-up (kernel attributes, device addresses of the
+ *     library's __device__ arrays) happens at the first call on a device and
+ *     is kept for the process; it does not survive cudaDeviceReset().
  *   - All calls are asynchronous on `stream` (a cudaStream_t; NULL is the
  *     legacy default stream).  None synchronises except fp8_get_status().
  *   - Arguments are validated on the host before anything is launched; on a
@@ -255,17 +258,47 @@ int fp8_moe_dispatch(const uint8_t* q, const float* sA, int64_t T, int64_t K, co
                      void* workspace, int64_t workspace_bytes, void* stream);
 
 /*
+ * 1x128 quantization of the tokens fused with their FP8 dispatch ([P5]
+ * hardware passage: 128 BF16 activations are read from HBM, quantized, the
+ * FP8 values written back and read again -- here the codes go straight to
+ * the expert-ordered rows; [P1]/[P3] dispatch in FP8; [P4] top-8 routing).
+ * Writes exactly what fp8_quant_act_1x128 followed by fp8_moe_dispatch
+ * writes into q_out, sA_out, group_offsets, token_row and row_token (the
+ * per-token codes q / sA are not produced).
+ *   x          [T][ldx] BF16 or FP32 tokens (in_dtype FP8_IN_*), row-major
+ *   scale_mode FP8_SCALE_FP32 or FP8_SCALE_POW2, as fp8_quant_act_1x128
+ *   the other arguments as fp8_moe_dispatch (same workspace size)
+ * Sizes: as fp8_moe_dispatch, plus ldx >= K and ldx * element size a
+ * multiple of 16 bytes; x 16-byte aligned.  Errors as fp8_moe_dispatch.
+ * Launches four kernels and one memset: the routing passes, the fused
+ * quantizer, and a pass that fills the padding rows.
+ */
+int fp8_moe_quant_dispatch(const void* x, int in_dtype, int64_t T, int64_t K, int64_t ldx,
+                           const int32_t* topk, int k, int G, uint8_t* q_out, float* sA_out,
+                           int64_t M_cap, int32_t* group_offsets, int32_t* token_row,
+                           int32_t* row_token, void* workspace, int64_t workspace_bytes,
+                           int scale_mode, void* stream);
+
+/*
  * fp8_moe_dispatch without a caller workspace: the same dispatch, writing
  * the same outputs, with its scratch in a fixed device array of
- * FP8_MOE_NOALLOC_WS_BYTES inside the library (one per device).  The pages
- * have no counterpart: this is an integration convenience for callers that
- * must not allocate (e.g. inside a CUDA graph), and it allocates nothing.
+ * FP8_MOE_NOALLOC_WS_BYTES inside the library (one per device, held by every
+ * device that loads the library until the process exits).  The pages have
+ * no counterpart.  It is for callers that cannot allocate device memory:
+ * code whose device memory is all handed out by a framework's own pool and
+ * that has no allocator to ask for scratch, and code that must not call
+ * cudaMalloc because cudaMalloc can synchronise the device in the middle of
+ * its queued work.  The call allocates nothing (no cudaMalloc, no library
+ * routine that allocates); the caller still passes inputs and outputs.
  *   Limit: fp8_moe_dispatch_workspace_bytes(T, k, G) <= FP8_MOE_NOALLOC_WS_BYTES
  *          (e.g. T*k <= 2^21 pairs at G = 32), else FP8_ERR_SHAPE.
- *   The first call on each device looks the array up (cudaGetSymbolAddress
- *   with that device current); make it before any stream capture.
+ *   Set-up: the first call in a CUDA context looks the array's device
+ *   address up (cudaGetSymbolAddress with the device current); a call from
+ *   another context looks it up again.  Make the first call before any
+ *   stream capture.
  *   Calls that overlap on one device (other streams, other threads) share
- *   the array and race: serialise them.  No clearing is needed between
+ *   the array and race: serialise them.  Every scratch entry a call reads is
+ *   written earlier in the same call, so nothing needs clearing between
  *   calls.  Other arguments, errors and launches as fp8_moe_dispatch.
  */
 #define FP8_MOE_NOALLOC_WS_BYTES 262144
@@ -313,6 +346,26 @@ void fp8_set_wait_timeout_ns(uint64_t ns);
  * usable.  Returns FP8_OK if the launch succeeded.
  */
 int fp8_selftest_wait_timeout(void* stream);
+
+/*
+ * Self-test of the GEMMs' unwinding after a wait runs out (no counterpart in
+ * the pages; it exercises the failure path of the kernels that do the work).
+ * Launches the promotion GEMM (kernel 0, fp8_blockscaled_gemm /
+ * fp8_grouped_gemm) or the tensor-core-scaled one (kernel 1,
+ * fp8_blockscaled_gemm_pow2 / fp8_grouped_gemm_pow2) -- grouped when
+ * group_offsets is not NULL -- with the odd CTA of every CTA pair holding
+ * back its operand loads after its first K-block.  The pair's MMA then waits
+ * for bytes that never come: the wait runs into its time limit
+ * (fp8_set_wait_timeout_ns), FP8_ERR_TIMEOUT is recorded in the status word,
+ * and every role of both CTAs unwinds (copies in flight drained, TMEM
+ * freed) and returns, leaving the context usable.  D is left partly written.
+ * Arguments as fp8_blockscaled_gemm with B K-major and per-block scales
+ * (ldd = N) or as fp8_grouped_gemm; K >= 256, so that a second K-block
+ * exists.  Returns FP8_OK if the launch succeeded.
+ */
+int fp8_selftest_gemm_unwind(int kernel, const uint8_t* A, const float* sA, const uint8_t* B,
+                             const float* sB, const int32_t* group_offsets, int G, int64_t M,
+                             int64_t N, int64_t K, void* D, int out_dtype, void* stream);
 
 /* 1 if the current device is an sm_100 GPU the library runs on, else 0. */
 int fp8_device_supported(void);

@@ -78,6 +78,7 @@ def test_dgrad_reads_weight_transposed():
     qdy, sdy = oracle.quant_act_1x128(_bits(wl["dy"]))
     qw, sw = oracle.quant_w_128x128(_bits(wl["w"]))               # stored [N_out][K_in]
     assert np.array_equal(step.qdy.cpu().numpy(), qdy) and np.array_equal(step.qw.cpu().numpy(), qw)
+    assert np.array_equal(step.sdy.cpu().numpy(), sdy) and np.array_equal(step.sw.cpu().numpy(), sw)
     M, N = dx.shape
     pts = _points(M, N, 2, rows=_edges(M, 128), cols=_edges(N, 256))
     ref, tol = oracle.gemm_points(qdy, sdy, qw, sw, pts, b_major=oracle.B_MNMAJOR)
@@ -170,9 +171,9 @@ def test_moe_grouped_fprop(pow2_tc):
     assert np.array_equal(off, lay.offsets.numpy())
     assert np.array_equal(step.row_token.cpu().numpy()[:lay.m_total], lay.row_token.numpy())
 
-    # tokens and weights quantized by the oracle, bit-exact
+    # weights quantized by the oracle, bit-exact; the tokens' codes exist
+    # only in their dispatched rows (checked below)
     qx, sx = oracle.quant_act_1x128(_bits(wl["x"]), mode)
-    assert np.array_equal(step.qx.cpu().numpy(), qx) and np.array_equal(step.sx.cpu().numpy(), sx)
     qw, sw = oracle.quant_w_128x128(_bits(wl["w"].view(G * N, K)), mode)
     assert np.array_equal(step.qw.cpu().numpy().reshape(G * N, K), qw)
     assert np.array_equal(step.sw.cpu().numpy().reshape(G * N // 128, K // 128), sw)

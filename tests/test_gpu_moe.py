@@ -75,6 +75,61 @@ def test_dispatch_reports_bad_expert_ids_and_overflow():
     assert fg.fp8_get_status() == fg.FP8_OK
 
 
+def _quant_dispatch(x, topk, G, mode, M_cap=None):
+    T, K = x.shape
+    k = topk.shape[1]
+    M_cap = fg.moe_capacity(T, k, G) if M_cap is None else M_cap
+    d = dev()
+    # outputs filled with junk, so that anything left unwritten shows
+    out = dict(q=torch.full((M_cap, K), 0x5A, dtype=torch.uint8, device=d),
+               sA=torch.full((K // 128, M_cap), -7.0, dtype=torch.float32, device=d),
+               offsets=torch.full((G + 1,), -9, dtype=torch.int32, device=d),
+               token_row=torch.full((T, k), -9, dtype=torch.int32, device=d),
+               row_token=torch.full((M_cap,), -9, dtype=torch.int32, device=d))
+    ws = torch.empty(max(1, fg.fp8_moe_dispatch_workspace_bytes(T, k, G) // 4), dtype=torch.int32,
+                     device=d)
+    fg.fp8_moe_quant_dispatch(x, to_dev(topk), G, out["q"], out["sA"], out["offsets"],
+                              out["token_row"], out["row_token"], ws, mode)
+    return out
+
+
+@pytest.mark.parametrize("T,K,k,G,dtype,mode", [
+    (1, 128, 1, 1, "bf16", fg.SCALE_POW2),
+    (300, 256, 4, 6, "bf16", fg.SCALE_FP32),       # ragged token count, an empty expert
+    (1000, 512, 8, 32, "fp32", fg.SCALE_POW2),
+    (129, 384, 20, 32, "bf16", fg.SCALE_FP32),     # more than 16 destinations per token
+])
+def test_quant_dispatch_equals_oracle_quantizer_then_dispatch(T, K, k, G, dtype, mode):
+    x = synth.activations(T, K, seed=T + k, outlier_seed=T + k + 1)
+    topk = synth.zipf_topk_routing(T, G, k, seed=T + G).numpy().astype(np.int32)
+    if G > 2:
+        topk[topk == G - 1] = 0                       # one expert receives nothing
+    xin = x if dtype == "bf16" else x.float()
+    got = _quant_dispatch(xin.to(dev()), topk, G, mode)
+    assert fg.fp8_get_status() == fg.FP8_OK
+    oq, os_ = oracle.quant_act_1x128(synth.bf16_bits(x) if dtype == "bf16" else xin.numpy(), mode)
+    ref = omoe.moe_dispatch(oq, os_, topk, G, got["q"].shape[0])
+    for key in ("offsets", "token_row", "row_token", "q"):
+        assert np.array_equal(got[key].cpu().numpy(), ref[key]), key
+    assert np.array_equal(got["sA"].cpu().numpy().view(np.uint32), ref["sA"].view(np.uint32))
+
+
+def test_quant_dispatch_reports_bad_expert_ids_like_the_dispatch():
+    T, K, k, G = 256, 256, 2, 4
+    x = synth.activations(T, K, seed=31, outlier_seed=32).to(dev())
+    topk = synth.zipf_topk_routing(T, G, k, seed=33).numpy().astype(np.int32)
+    topk[5, 1] = 4                                    # outside [0, G)
+    got = _quant_dispatch(x, topk, G, fg.SCALE_FP32)
+    assert fg.fp8_get_status() == fg.FP8_ERR_SHAPE
+    assert got["token_row"][5, 1].item() == -1
+    qx, sx = fg.quant_act_1x128(x)
+    ref = fg.moe_dispatch(qx, sx, to_dev(topk), G)
+    assert fg.fp8_get_status() == fg.FP8_ERR_SHAPE
+    for key in ("offsets", "token_row", "row_token", "q"):
+        assert torch.equal(got[key], ref[key]), key
+    assert torch.equal(got["sA"].view(torch.int32), ref["sA"].view(torch.int32))
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
 def test_combine_matches_oracle(dtype):
     rng = np.random.default_rng(3)

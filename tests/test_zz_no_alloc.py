@@ -37,8 +37,11 @@ def _outputs(T, K, k, G):
 @pytest.mark.gpu
 def test_noalloc_dispatch_equals_workspace_dispatch_twice_in_a_row():
     # the second case has a different expert count and chunk count, so scratch
-    # left over from the first call would change its result
-    for (T, K, k, G, seed) in [(3000, 512, 8, 32, 41), (1000, 256, 4, 6, 43)]:
+    # left over from the first call would change its result; the third fills
+    # the fixed scratch exactly (64 chunks of 1024 pairs x 1024 experts)
+    cases = [(3000, 512, 8, 32, 41), (1000, 256, 4, 6, 43), (8192, 128, 8, 1024, 47)]
+    assert fg.fp8_moe_dispatch_workspace_bytes(8192, 8, 1024) == 262144
+    for (T, K, k, G, seed) in cases:
         q, sA, topk = _case(T, K, k, G, seed)
         ref = _outputs(T, K, k, G)
         ws = torch.empty(max(1, fg.fp8_moe_dispatch_workspace_bytes(T, k, G) // 4),
