@@ -191,6 +191,18 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void*
                  : "memory");
 }
 
+// The same box added element-wise into global memory (the tensor map's type
+// must be one the TMA adds, e.g. FP32).
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const void* smem_src,
+                                                  int32_t x, int32_t y)
+{
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(x), "r"(y), "r"(smem_u32(smem_src))
+        : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 // Wait until at most N of this thread's bulk groups still read shared memory.
@@ -484,6 +496,12 @@ __device__ __forceinline__ void pair_block_offsets(const int32_t* off, int32_t* 
 // driver's encoder is unavailable).
 bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128 = true);
+
+// Host: 2-D tensor map of `dtype` elements [outer][inner] (inner in
+// elements), rows `row_bytes` apart, boxes of box_inner x box_outer elements,
+// no swizzle (defined in gemm.cu).
+bool make_map_typed(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                    uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
 
 // ---------------------------------------------------------------- registers
 

@@ -67,7 +67,7 @@ constexpr int NUM_THREADS = 128 + 32 * NUM_PROMO_WARPS; // 384 = 3 warpgroups
 // down to 8); warpgroup 0 (TMA, MMA, 2 idle warps) drops to CTRL_REGS and the
 // two promotion warpgroups rise to PROMO_REGS, within the launch total.
 constexpr uint32_t LAUNCH_REGS = 168;
-constexpr uint32_t CTRL_REGS = 40;
+constexpr uint32_t CTRL_REGS = 72;
 constexpr uint32_t PROMO_REGS = 216;
 static_assert(128 * CTRL_REGS + 256 * PROMO_REGS <= NUM_THREADS * LAUNCH_REGS,
               "register split exceeds the launch allocation");
@@ -89,6 +89,7 @@ struct GemmParams {
     int G;
     int b_major, sb_gran, out_dtype;
     int band;                      // m-blocks per raster band
+    int streamk;                   // 1: contiguous ranges of (tile, K-block) units per pair
     int withhold;                  // self-test: the odd CTA stops loading after one K-block
     uint64_t timeout_ns;
 };
@@ -135,11 +136,61 @@ __device__ __forceinline__ bool tile_rows(const GemmParams& p, const Shared& sh,
     return tile_rows(p.group_offsets, sh.off, sh.poff, p.G, p.M, mb, rank, t);
 }
 
-// Tiles are dealt round-robin to pairs: pair c is CTAs 2c, 2c+1.
-__device__ __forceinline__ void unit_range(int64_t& first, int64_t& stride)
+// The work of pair c (CTAs 2c, 2c+1) as a sequence of segments: a tile and
+// the range [kb0, kb1) of its K-blocks.  Normally tiles are dealt round-robin
+// and every segment is a whole tile.  With stream-K the tiles' K-blocks are
+// laid end to end (tile t owns units t*nkb .. t*nkb+nkb-1) and pair c takes
+// the contiguous units [c*U/P, (c+1)*U/P): every pair gets the same work, and
+// a tile cut between two pairs has exactly two contributors (each range is
+// at least one tile long), which add their partial sums into D.
+struct Segments {
+    int64_t tile, kb0, kb1;   // current segment
+    int64_t u, u_end;         // stream-K: next unit, end of this pair's range
+    int64_t stride;           // round-robin: tiles between this pair's tiles
+    int64_t ntiles, nkb;
+    bool streamk;
+};
+
+__device__ __forceinline__ void seg_set(Segments& g)
 {
-    first = (int64_t)(blockIdx.x >> 1);
-    stride = (int64_t)(gridDim.x >> 1);
+    g.tile = g.u / g.nkb;
+    g.kb0 = g.u - g.tile * g.nkb;
+    const int64_t left = g.u_end - g.u;
+    g.kb1 = g.kb0 + left < g.nkb ? g.kb0 + left : g.nkb;
+}
+
+__device__ __forceinline__ void seg_begin(Segments& g, const GemmParams& p, int64_t ntiles,
+                                          int64_t nkb)
+{
+    const int64_t pair = (int64_t)(blockIdx.x >> 1), pairs = (int64_t)(gridDim.x >> 1);
+    g.ntiles = ntiles;
+    g.nkb = nkb;
+    g.streamk = p.streamk != 0;
+    if (g.streamk) {
+        const int64_t units = ntiles * nkb;
+        g.u = pair * units / pairs;
+        g.u_end = (pair + 1) * units / pairs;
+        if (g.u < g.u_end) seg_set(g);
+        else g.tile = ntiles;
+    } else {
+        g.stride = pairs;
+        g.tile = pair;
+        g.kb0 = 0;
+        g.kb1 = nkb;
+    }
+}
+
+__device__ __forceinline__ bool seg_valid(const Segments& g) { return g.tile < g.ntiles; }
+
+__device__ __forceinline__ void seg_next(Segments& g)
+{
+    if (g.streamk) {
+        g.u += g.kb1 - g.kb0;
+        if (g.u < g.u_end) seg_set(g);
+        else g.tile = g.ntiles;
+    } else {
+        g.tile += g.stride;
+    }
 }
 
 __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const GemmParams& p,
@@ -149,11 +200,10 @@ __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, con
     const uint32_t rank = cluster_ctarank();
     int64_t it = 0;   // loads issued so far; stage it % NS, round it / NS
     bool ok = true;
-    int64_t first, stride;
-    unit_range(first, stride);
-    for (int64_t tile = first; ok && tile < nmb * nnb; tile += stride) {
+    Segments sg;
+    for (seg_begin(sg, p, nmb * nnb, nkb); ok && seg_valid(sg); seg_next(sg)) {
         int64_t mb, nb;
-        gemm_tile_coord(tile, nmb, nnb, p.band, mb, nb);
+        gemm_tile_coord(sg.tile, nmb, nnb, p.band, mb, nb);
         TileRows tr;
         if (!tile_rows(p, sh, mb, rank, tr)) continue;
         // (an idle odd CTA still loads its rows: the pair's MMA counts them)
@@ -163,7 +213,7 @@ __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, con
         // A CTA of a pair loads B's columns rank*128 .. rank*128+127 of the
         // tile (a box counts in full, its out-of-range part zero-filled).
         const int32_t brow = (int32_t)((int64_t)g * p.N + n0 + rank * 128);
-        for (int64_t kb = 0; kb < nkb; ++kb) {
+        for (int64_t kb = sg.kb0; kb < sg.kb1; ++kb) {
             if (p.withhold && rank == 1 && it == 1) {   // self-test only
                 ok = false;
                 break;
@@ -209,16 +259,11 @@ __device__ void run_mma(const GemmParams& p, uint8_t* smem, Shared& sh, int64_t 
     const uint32_t tmem = sh.tmem_base;
     int64_t it = 0, kbg = 0;
     bool ok = true;
-    int64_t first, stride;
-    unit_range(first, stride);
-    for (int64_t tile = first; ok && tile < nmb * nnb; tile += stride) {
-        int64_t mb, nb;
-        gemm_tile_coord(tile, nmb, nnb, p.band, mb, nb);
-        (void)mb;
-        (void)nb;
+    Segments sg;
+    for (seg_begin(sg, p, nmb * nnb, nkb); ok && seg_valid(sg); seg_next(sg)) {
         // A pair's MMA always spans 256 columns (a B tail is zero-filled).
         const uint32_t idesc = idesc_e4m3_f32((uint32_t)TILE_M, (uint32_t)BN, (uint32_t)p.b_major);
-        for (int64_t kb = 0; kb < nkb; ++kb, ++it, ++kbg) {
+        for (int64_t kb = sg.kb0; kb < sg.kb1; ++kb, ++it, ++kbg) {
             const int s = (int)(it % NS);
             const uint32_t ph = (uint32_t)((it / NS) & 1);
             const uint32_t buf = (uint32_t)(kbg & 1);
@@ -264,11 +309,14 @@ __device__ void run_promotion(const CUtensorMap* tmD, const GemmParams& p, Share
     const int nnb128 = (int)(p.N / 128);
     uint32_t kbg = 0;
 
-    int64_t first, stride;
-    unit_range(first, stride);
-    for (int tile = (int)first; tile < nmb * nnb; tile += (int)stride) {
+    Segments sg;
+    for (seg_begin(sg, p, (int64_t)nmb * nnb, nkb); seg_valid(sg); seg_next(sg)) {
         int64_t mb64, nb64;
-        gemm_tile_coord(tile, nmb, nnb, p.band, mb64, nb64);
+        gemm_tile_coord(sg.tile, nmb, nnb, p.band, mb64, nb64);
+        const int kb0 = (int)sg.kb0, kb1 = (int)sg.kb1;
+        // the whole K range of the tile (a plain store), or a stream-K part
+        // of it (the two parts are added into D, which starts at zero)
+        const bool whole = kb0 == 0 && kb1 == nkb;
         TileRows tr;
         if (!tile_rows(p, sh, mb64, (uint32_t)rank, tr)) continue;
         const int nb = (int)nb64;
@@ -286,22 +334,23 @@ __device__ void run_promotion(const CUtensorMap* tmD, const GemmParams& p, Share
         //   sb   its 128-column block's weight scale (sb_gran 128), or
         //   sb4  4 of its half's 128 column scales (sb_gran 1), staged in this
         //        warp's shared buffer so every lane can read all 128.
-        const float* sa_ptr = p.sA + (row_ok ? m : 0);
+        const float* sa_ptr = p.sA + (row_ok ? m + (int64_t)kb0 * p.M : 0);
         const int64_t sa_step = row_ok ? p.M : 0;
         const bool use_sb = active && p.sb_gran == 128;
         const float* sb_ptr = p.sB;
         int64_t sb_step = 0;
         if (p.sb_gran == 128) {
             if (p.b_major == FP8_B_KMAJOR) {
-                sb_ptr = p.sB + ((int64_t)g * nnb128 + cb) * nkb;
+                sb_ptr = p.sB + ((int64_t)g * nnb128 + cb) * nkb + kb0;
                 sb_step = 1;
             } else {
-                sb_ptr = p.sB + cb;
+                sb_ptr = p.sB + cb + (int64_t)kb0 * nnb128;
                 sb_step = nnb128;
             }
         }
         const bool use_sb4 = active && p.sb_gran == 1;
-        const float4* sb4_ptr = reinterpret_cast<const float4*>(p.sB + n0 + col0) + lane;
+        const float4* sb4_ptr =
+            reinterpret_cast<const float4*>(p.sB + (int64_t)kb0 * p.N + n0 + col0) + lane;
         const int64_t sb4_step = p.N / 4;
 
         float acc[128];
@@ -311,15 +360,15 @@ __device__ void run_promotion(const CUtensorMap* tmD, const GemmParams& p, Share
         float sa_next = row_ok ? __ldg(sa_ptr) : 0.0f;
         float sb_next = use_sb ? __ldg(sb_ptr) : 0.0f;
         if (p.sb_gran == 1) {
-            *reinterpret_cast<float4*>(&sh.sbw[ew][0][lane * 4]) =
+            *reinterpret_cast<float4*>(&sh.sbw[ew][kb0 & 1][lane * 4]) =
                 use_sb4 ? __ldg(sb4_ptr) : make_float4(0.f, 0.f, 0.f, 0.f);
             __syncwarp();
         }
         bool ok = true;
-        for (int kb = 0; kb < nkb; ++kb, ++kbg) {
+        for (int kb = kb0; kb < kb1; ++kb, ++kbg) {
             const float sa = sa_next, sb = sb_next;
             float4 sb4_next = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (kb + 1 < nkb) {
+            if (kb + 1 < kb1) {
                 sa_ptr += sa_step;
                 sb_ptr += sb_step;
                 sb4_ptr += sb4_step;
@@ -396,14 +445,16 @@ __device__ void run_promotion(const CUtensorMap* tmD, const GemmParams& p, Share
 
         // Epilogue: round the FP32 sums to the output type and store them.
         // Each lane writes its row's next 32 bytes into this warp's staging
-        // buffer; one lane hands the 32 x 32-byte box to a TMA store, which
-        // drops the rows beyond M and the columns beyond N.  Two buffers
-        // alternate, so a store's read of one overlaps the writes of the other.
+        // buffer; one lane hands the 32 x 32-byte box to a TMA store (or, for
+        // a stream-K part of a tile, a TMA reduce-add), which drops the rows
+        // beyond M and the columns beyond N.  Two buffers alternate, so a
+        // store's read of one overlaps the writes of the other.
         if (active) {
             const int esz = p.out_dtype == FP8_OUT_BF16 ? 2 : 4;
             const int nch = 128 * esz / EPI_BYTES;                 // 8 (BF16) or 16 (FP32)
             const int32_t y = m0 + quad * 32;
-            const int32_t x0 = (n0 + col0) * esz;
+            const int32_t x0 = n0 + col0;                          // elements
+            const int xstep = EPI_BYTES / esz;
 #pragma unroll
             for (int ch = 0; ch < 16; ++ch) {
                 if (ch >= nch) break;
@@ -429,7 +480,10 @@ __device__ void run_promotion(const CUtensorMap* tmD, const GemmParams& p, Share
                 fence_proxy_async_shared();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_2d(tmD, buf, x0 + ch * EPI_BYTES, y);
+                    if (whole)
+                        tma_store_2d(tmD, buf, x0 + ch * xstep, y);
+                    else   // stream-K part of an FP32 tile: add into D
+                        tma_reduce_add_2d(tmD, buf, x0 + ch * xstep, y);
                     bulk_commit_group();
                 }
             }
@@ -631,7 +685,44 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_map_typed(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                    uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 namespace {
+
+// Zero the tiles that stream-K splits between two pairs (the tile holding
+// the first unit of each pair's range, when that unit is not a tile's
+// first): their two parts are added into D.  CTA c handles pair c's tile,
+// 256 threads over its 256 rows x 256 FP32 columns (clipped to M and N).
+__global__ void __launch_bounds__(256) k_zero_split_tiles(float* __restrict__ D, int64_t ldd,
+                                                          int64_t M, int64_t N, int64_t nmb,
+                                                          int64_t nnb, int64_t nkb, int64_t pairs,
+                                                          int band)
+{
+    const int64_t units = nmb * nnb * nkb;
+    const int64_t u = (int64_t)blockIdx.x * units / pairs;
+    if (blockIdx.x == 0 || u % nkb == 0) return;
+    int64_t mb, nb;
+    gemm_tile_coord(u / nkb, nmb, nnb, band, mb, nb);
+    const int64_t r0 = mb * TILE_M, c0 = nb * BN;
+    const int64_t rows = M - r0 < TILE_M ? M - r0 : TILE_M;
+    const int64_t cols = N - c0 < BN ? N - c0 : BN;
+    for (int64_t i = threadIdx.x; i < rows * (cols / 4); i += blockDim.x) {
+        const int64_t r = i / (cols / 4), c = (i % (cols / 4)) * 4;
+        *reinterpret_cast<float4*>(D + (r0 + r) * ldd + c0 + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
 
 int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, int b_major, const float* sB,
                 int sb_gran, int64_t M, int64_t N, int64_t K, const int32_t* group_offsets, int G,
@@ -653,10 +744,12 @@ int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, int b_major
     if (!okB) return FP8_ERR_LAUNCH;
     // D as bytes: rows of N * element-size bytes, `ldd` elements apart; the
     // epilogue stores 32-byte x 32-row boxes
+    // D in its element type; the epilogue stores boxes of 32 bytes x 32 rows
     CUtensorMap tmD;
-    const uint64_t esz = out_dtype == FP8_OUT_BF16 ? 2 : 4;
-    if (!make_map(&tmD, D, (uint64_t)N * esz, (uint64_t)M, (uint64_t)ldd * esz, EPI_BYTES, EPI_ROWS,
-                  false))
+    const bool bf16 = out_dtype == FP8_OUT_BF16;
+    const uint32_t esz = bf16 ? 2 : 4;
+    if (!make_map_typed(&tmD, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                        D, (uint64_t)N, (uint64_t)M, (uint64_t)ldd * esz, EPI_BYTES / esz, EPI_ROWS))
         return FP8_ERR_LAUNCH;
     GemmParams p;
     p.sA = sA;
@@ -675,8 +768,23 @@ int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, int b_major
     p.band = group_offsets ? BAND_GROUPED : BAND_DENSE;
     p.timeout_ns = wait_timeout_ns();
     // grouped: each group adds at most one partly idle 256-row block
-    const int64_t tiles = ((M + 255) / 256 + (group_offsets ? G : 0)) * ((N + BN - 1) / BN);
+    const int64_t nnb = (N + BN - 1) / BN, nkb = K / BK;
+    const int64_t tiles = ((M + 255) / 256 + (group_offsets ? G : 0)) * nnb;
     const int64_t clusters = tiles < setup.pair_clusters ? tiles : setup.pair_clusters;
+    // Stream-K for dense FP32 outputs whose tiles fill the last round of the
+    // pairs badly (the parts of a split tile are added exactly: two FP32
+    // sums onto zero, in either order, give the same result).  Each pair's
+    // range must hold at least a whole tile, so that no tile has more than
+    // two contributors.
+    const int64_t rounds = (tiles + clusters - 1) / clusters;
+    p.streamk = !bf16 && !group_offsets && tiles > clusters && tiles % clusters != 0 &&
+                (double)rounds * clusters / (double)tiles > 1.05 && tiles * nkb / clusters >= nkb;
+    if (p.streamk) {
+        const int64_t nmb = (M + TILE_M - 1) / TILE_M;
+        k_zero_split_tiles<<<(unsigned)clusters, 256, 0, st>>>(static_cast<float*>(D), ldd, M, N,
+                                                              nmb, nnb, nkb, clusters, p.band);
+        if (cudaGetLastError() != cudaSuccess) return FP8_ERR_LAUNCH;
+    }
     cudaLaunchAttribute attr[1];
     const cudaLaunchConfig_t cfg = pair_launch_config((unsigned)clusters, st, attr);
     return cudaLaunchKernelEx(&cfg, k_fp8_gemm, tmA, tmB, tmD, p) == cudaSuccess ? FP8_OK

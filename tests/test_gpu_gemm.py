@@ -180,3 +180,18 @@ def test_bounded_wait_times_out_and_context_survives():
 
 def test_device_supported():
     assert fg.fp8_device_supported()
+
+
+@pytest.mark.parametrize("sb_gran", [128, 1])
+def test_stream_k_fp32_output_matches_oracle_and_is_deterministic(sb_gran):
+    # 10 x 8 = 80 pair tiles on 74 pairs: the FP32 GEMM splits its K-blocks
+    # evenly over the pairs, so tiles cut between two pairs get their two
+    # parts added into D.  The sum of two FP32 parts onto zero does not depend
+    # on their order: two runs give identical bits.
+    M, N, K = 2560, 2048, 512
+    A, sA, B, sB = _operands(M, N, K, fg.B_KMAJOR, sb_gran, seed=77)
+    got = _run(A, sA, B, sB, fg.B_KMAJOR, sb_gran, torch.float32)
+    again = _run(A, sA, B, sB, fg.B_KMAJOR, sb_gran, torch.float32)
+    assert np.array_equal(got.view(np.uint64), again.view(np.uint64))
+    ref, tol = oracle.gemm_full(A, sA, B, sB, sb_gran=sb_gran)
+    assert_gemm_close(got, ref, tol, False, f"stream-K sb_gran={sb_gran}")
