@@ -128,12 +128,22 @@ def gemm_kernel(workload: str) -> str:
     return "k_fp8_gemm_mx" if workload.endswith("_tc") else "k_fp8_gemm"
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source without comments, trailing blanks and empty lines, so
+    that a comment edit does not invalidate a capture of the same code."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def kernel_source_hash(kernel: str = "k_fp8_gemm") -> str:
+    """sha256 (first 16 hex digits) of the kernel's sources, comments removed."""
     import hashlib
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

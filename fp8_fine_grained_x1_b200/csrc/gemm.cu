@@ -21,7 +21,9 @@
 //               to the promotion warpgroups)
 //   warps 4-11  promotion + epilogue: tcgen05.ld the partial, FMA it (packed
 //               FP32x2) with its scale into a register accumulator, release the
-//               buffer; after the last K-block convert to BF16/FP32 and store.
+//               buffer; after the last K-block convert to BF16/FP32, stage 32
+//               rows x 32 bytes at a time in shared memory and hand them to a
+//               TMA store, then go on with the next tile at once.
 // Each CTA promotes a 128 (M) x 256 (N) block; warps 4-7 own its columns
 // 0-127, warps 8-11 columns 128-255, each warp the 32 TMEM lanes (rows) its
 // id allows.
@@ -37,6 +39,12 @@
 // their 256-row blocks group by group, so that both halves of a pair use the
 // same expert's B; a group of an odd number of 128-row blocks leaves the odd
 // CTA of its last pair idle.
+//
+// Work is dealt to the pairs tile by tile, in raster bands of M-blocks.  For
+// FP32 outputs whose tile count leaves the last round poorly filled, the
+// pairs instead take equal contiguous ranges of (tile, K-block) units
+// (stream-K): a tile cut between two pairs gets two partial sums, which TMA
+// reduce-adds into D after a small kernel has zeroed those tiles.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -97,7 +105,7 @@ struct GemmParams {
 
 // Epilogue staging: each promotion warp writes its 32 rows x 32 bytes of
 // output at a time into one of two 1 KB buffers, from which a TMA store
-// copies them to D (EPI_COLS_B bytes wide, 32 rows).
+// copies them to D (boxes EPI_BYTES wide, EPI_ROWS rows).
 constexpr int EPI_BYTES = 32;                           // bytes of a row per store
 constexpr int EPI_ROWS = 32;
 

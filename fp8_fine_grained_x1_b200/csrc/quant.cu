@@ -70,14 +70,24 @@ __device__ __forceinline__ GroupScale group_scale(float amax, int mode)
     return g;
 }
 
-// Four scaled values -> four E4M3 codes packed little-endian in a uint32.
+// Four scaled values -> four E4M3 codes packed little-endian in a uint32:
+// byte i = E4M3(fl32(x_i * inv)), round to nearest even, saturating to
+// +-448.  The products are two packed FP32x2 multiplies (each lane rounded
+// to nearest like a scalar multiply); each cvt packs two codes, its first
+// source going to the upper byte.
 __device__ __forceinline__ uint32_t encode4(float a, float b, float c, float d, float inv)
 {
-    const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
-        make_float2(__fmul_rn(a, inv), __fmul_rn(b, inv)), __NV_SATFINITE, __NV_E4M3);
-    const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
-        make_float2(__fmul_rn(c, inv), __fmul_rn(d, inv)), __NV_SATFINITE, __NV_E4M3);
-    return (uint32_t)lo | ((uint32_t)hi << 16);
+    float a2, b2, c2, d2;
+    fmul2(a2, b2, a, b, inv, inv);
+    fmul2(c2, d2, c, d, inv, inv);
+    uint32_t r;
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+        "mov.b32 %0, {lo, hi};\n\t}"
+        : "=r"(r)
+        : "f"(a2), "f"(b2), "f"(c2), "f"(d2));
+    return r;
 }
 
 // ------------------------------------------------------------ vector loads
@@ -474,8 +484,8 @@ __global__ void __launch_bounds__(kThr128x1, 5) k_quant_128x1(const Tin* __restr
 
 // Activations cached as 1x128 E4M3 tiles (the forward pass's quantized X)
 // regrouped for the Wgrad GEMM: every code is dequantized to
-// fl32(decode(q) * sA) -- E4M3 -> FP16 -> FP32 is exact, so __fmul_rn gives
-// that single rounding -- and the FP32 values are quantized in 128x1 groups
+// fl32(decode(q) * sA) -- E4M3 -> FP16 -> FP32 is exact, so one FP32
+// multiply gives that single rounding -- and the FP32 values are quantized in 128x1 groups
 // along tokens, exactly as k_quant_128x1 quantizes an FP32 input.
 //
 // CTA = 256 threads over kReqTiles consecutive tiles of 128 tokens x 128
@@ -485,7 +495,8 @@ __global__ void __launch_bounds__(kThr128x1, 5) k_quant_128x1(const Tin* __restr
 // tokens 16w .. 16w+15 and lane l channels 4l .. 4l+3, read as one 32-bit
 // word per token (a warp reads a whole 128-byte row, conflict-free).
 // Pass 1: dequantize once (the 64 products stay in registers) and take the
-// max-abs, combined over the 8 warps through shared memory.  Pass 2: each
+// max-abs, combined over the 8 warps through shared memory, where thread c
+// (c < 128) derives channel c's scale once for the CTA.  Pass 2: each
 // thread encodes its 16 tokens of each of its 4 channels into one 16-byte
 // word.  The staged tile is dead by then, so the transposed codes go
 // back into the same buffer (16-byte chunks XOR-swizzled by (channel / 4) %
@@ -495,13 +506,22 @@ constexpr int kReqTok = 128;
 constexpr int kReqCh = 128;
 constexpr int kReqTiles = 4;
 
+// Four E4M3 codes (little-endian in w) -> their exact values: each pair of
+// codes widens to FP16x2 (exact: E4M3 is a subset of FP16), each FP16 to FP32.
 __device__ __forceinline__ void decode4_e4m3(uint32_t w, float (&f)[4])
 {
-    const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xFFFFu), __NV_E4M3);
-    const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w >> 16), __NV_E4M3);
-    const float2 a = __half22float2(__half2(lo));
-    const float2 b = __half22float2(__half2(hi));
-    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+    asm("{\n\t.reg .b16 q0, q1, h0, h1, h2, h3;\n\t.reg .b32 p0, p1;\n\t"
+        "mov.b32 {q0, q1}, %4;\n\t"
+        "cvt.rn.f16x2.e4m3x2 p0, q0;\n\t"
+        "cvt.rn.f16x2.e4m3x2 p1, q1;\n\t"
+        "mov.b32 {h0, h1}, p0;\n\t"
+        "mov.b32 {h2, h3}, p1;\n\t"
+        "cvt.f32.f16 %0, h0;\n\t"
+        "cvt.f32.f16 %1, h1;\n\t"
+        "cvt.f32.f16 %2, h2;\n\t"
+        "cvt.f32.f16 %3, h3;\n\t}"
+        : "=f"(f[0]), "=f"(f[1]), "=f"(f[2]), "=f"(f[3])
+        : "r"(w));
 }
 
 __global__ void __launch_bounds__(256, 3) k_requant_128x1(const uint8_t* __restrict__ q, int64_t ldq,
@@ -511,6 +531,7 @@ __global__ void __launch_bounds__(256, 3) k_requant_128x1(const uint8_t* __restr
 {
     __shared__ __align__(16) uint8_t tile[2][kReqTok * kReqCh];   // codes, then transposed codes
     __shared__ __align__(16) float part[8][kReqCh];
+    __shared__ __align__(16) float inv_s[kReqCh];   // per-channel encode factors of the tile
     __shared__ float scl[2][kReqTok];
 
     const int64_t cb = blockIdx.x;
@@ -555,23 +576,25 @@ __global__ void __launch_bounds__(256, 3) k_requant_128x1(const uint8_t* __restr
             float f[4];
             decode4_e4m3(tw[t * (kReqCh / 4) + lane], f);
             const float sc = sc_t[t];
+            fmul2(v[i][0], v[i][1], f[0], f[1], sc, sc);
+            fmul2(v[i][2], v[i][3], f[2], f[3], sc, sc);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                v[i][k] = __fmul_rn(f[k], sc);
-                a[k] = fmaxf(a[k], fabsf(v[i][k]));
-            }
+            for (int k = 0; k < 4; ++k) a[k] = fmaxf(a[k], fabsf(v[i][k]));
         }
         *reinterpret_cast<float4*>(&part[w][4 * lane]) = make_float4(a[0], a[1], a[2], a[3]);
         __syncthreads();
+        if (threadIdx.x < kReqCh) {   // channel c = threadIdx.x: combine the warps, derive its scale
+            const int c = threadIdx.x;
+            float am = part[0][c];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const float4 pv = *reinterpret_cast<const float4*>(&part[k][4 * lane]);
-            a[0] = fmaxf(a[0], pv.x); a[1] = fmaxf(a[1], pv.y);
-            a[2] = fmaxf(a[2], pv.z); a[3] = fmaxf(a[3], pv.w);
+            for (int k = 1; k < 8; ++k) am = fmaxf(am, part[k][c]);
+            const GroupScale gs = group_scale(am, mode);
+            inv_s[c] = gs.inv;
+            s[tb * C + c0 + c] = gs.s;
         }
-        GroupScale g[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) g[k] = group_scale(a[k], mode);
+        __syncthreads();   // inv_s is ready; every read of the staged codes is done
+        const float4 inv4 = *reinterpret_cast<const float4*>(&inv_s[4 * lane]);
+        const float inv[4] = {inv4.x, inv4.y, inv4.z, inv4.w};
 
         // pass 2: encode 16 tokens x 4 channels into four 16-byte words
         uint32_t out[4][4];
@@ -580,9 +603,8 @@ __global__ void __launch_bounds__(256, 3) k_requant_128x1(const uint8_t* __restr
 #pragma unroll
             for (int k = 0; k < 4; ++k)
                 out[k][q4] = encode4(v[4 * q4][k], v[4 * q4 + 1][k], v[4 * q4 + 2][k], v[4 * q4 + 3][k],
-                                     g[k].inv);
+                                     inv[k]);
         }
-        __syncthreads();   // every read of the staged codes and of part is done
         uint8_t* tl = tile[buf];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -590,10 +612,6 @@ __global__ void __launch_bounds__(256, 3) k_requant_128x1(const uint8_t* __restr
             const int chunk = w ^ (lane & 7);
             *reinterpret_cast<uint4*>(&tl[c * kReqTok + chunk * 16]) =
                 make_uint4(out[k][0], out[k][1], out[k][2], out[k][3]);
-        }
-        if (w == 0) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) s[tb * C + c0 + 4 * lane + k] = g[k].s;
         }
         __syncthreads();
         const int64_t t0 = tb * kReqTok;

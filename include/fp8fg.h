@@ -294,8 +294,7 @@ int fp8_moe_quant_dispatch(const void* x, int in_dtype, int64_t T, int64_t K, in
  *          (e.g. T*k <= 2^21 pairs at G = 32), else FP8_ERR_SHAPE.
  *   Set-up: the first call in a CUDA context looks the array's device
  *   address up (cudaGetSymbolAddress with the device current); a call from
- *   another context looks it up again.  Make the first call before any
- *   stream capture.
+ *   another context looks it up again.
  *   Calls that overlap on one device (other streams, other threads) share
  *   the array and race: serialise them.  Every scratch entry a call reads is
  *   written earlier in the same call, so nothing needs clearing between
