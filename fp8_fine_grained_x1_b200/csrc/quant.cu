@@ -532,7 +532,7 @@ __global__ void __launch_bounds__(256, 3) k_requant_128x1(const uint8_t* __restr
     __shared__ __align__(16) uint8_t tile[2][kReqTok * kReqCh];   // codes, then transposed codes
     __shared__ __align__(16) float part[8][kReqCh];
     __shared__ __align__(16) float inv_s[kReqCh];   // per-channel encode factors of the tile
-    __shared__ float scl[2][kReqTok];
+    __shared__ __align__(16) float scl[2][kReqTok];
 
     const int64_t cb = blockIdx.x;
     const int64_t c0 = cb * kReqCh;
@@ -570,16 +570,20 @@ __global__ void __launch_bounds__(256, 3) k_requant_128x1(const uint8_t* __restr
         const float* sc_t = scl[buf];
         float v[16][4];
         float a[4] = {0.f, 0.f, 0.f, 0.f};
+        // tokens are taken in pairs (i, i+1): one packed multiply scales the
+        // same channel of both, the pairing the encode below uses as well
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < 16; i += 2) {
             const int t = w * 16 + i;
-            float f[4];
-            decode4_e4m3(tw[t * (kReqCh / 4) + lane], f);
-            const float sc = sc_t[t];
-            fmul2(v[i][0], v[i][1], f[0], f[1], sc, sc);
-            fmul2(v[i][2], v[i][3], f[2], f[3], sc, sc);
+            float f0[4], f1[4];
+            decode4_e4m3(tw[t * (kReqCh / 4) + lane], f0);
+            decode4_e4m3(tw[(t + 1) * (kReqCh / 4) + lane], f1);
+            const float2 sc = *reinterpret_cast<const float2*>(&sc_t[t]);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) a[k] = fmaxf(a[k], fabsf(v[i][k]));
+            for (int k = 0; k < 4; ++k) {
+                fmul2(v[i][k], v[i + 1][k], f0[k], f1[k], sc.x, sc.y);
+                a[k] = fmaxf(a[k], fmaxf(fabsf(v[i][k]), fabsf(v[i + 1][k])));
+            }
         }
         *reinterpret_cast<float4*>(&part[w][4 * lane]) = make_float4(a[0], a[1], a[2], a[3]);
         __syncthreads();
