@@ -103,6 +103,19 @@ def gemm_roofline(gemm_tflops: float, clocks: dict, peaks: dict) -> dict:
     return out
 
 
+def targets(roof: dict, quant_gbs: float) -> dict:
+    """The two targets of the path and the fraction each is judged on: the
+    GEMM against the dense FP8 spec (4.5 PFLOP/s, >= 60 %), the quantizers
+    against the HBM spec (8 TB/s, >= 75 %).  The measured-peak fractions in
+    `roofline` and `quantizers` are the engineering view beside them."""
+    g = roof["achieved"] / FP8_SPEC_TFLOPS
+    q = quant_gbs / HBM_SPEC_GBS
+    return {"gemm": {"judged_on": f"achieved / {FP8_SPEC_TFLOPS} TFLOP/s dense FP8 spec",
+                     "frac": g, "threshold": 0.60, "met": g >= 0.60},
+            "quantizers": {"judged_on": f"achieved / {HBM_SPEC_GBS} GB/s HBM spec",
+                           "frac": q, "threshold": 0.75, "met": q >= 0.75}}
+
+
 def run_config(desc: dict, world: int, host_inputs) -> dict:
     """The config object of the JSON line (both arms print the same one)."""
     cfg = dict(desc)
@@ -608,6 +621,7 @@ def main():
                            "frac_spec": quant_gbs / HBM_SPEC_GBS, "ms_per_step": quant_avg,
                            "algorithmic_bytes": quant_bytes},
             "gemm_ms": gemm_avg, "gemm_ms_min": gemm_ms[0],
+            "targets": targets(roof, quant_gbs),
             "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": step.kernel_calls * args.steps,
             "clocks": clock_summary,
