@@ -278,7 +278,7 @@ FP8FG_API int fp8_moe_quant_dispatch(const void* x, int in_dtype, int64_t T, int
             cudaSuccess ||
         launch_quant_act_1x128_dispatch(x, in_dtype, T, K, ldx, token_row, k, M_cap, q_out,
                                         sA_out, scale_mode, st) != cudaSuccess ||
-        launch_moe_rows(nullptr, nullptr, T, K, row_token, M_cap, q_out, sA_out, true, st) !=
+        launch_moe_pad_rows(group_offsets, G, K, row_token, M_cap, q_out, sA_out, st) !=
             cudaSuccess)
         return FP8_ERR_LAUNCH;
     return FP8_OK;

@@ -48,13 +48,16 @@ cudaError_t launch_moe_dispatch(const uint8_t* q, const float* sA, int64_t T, in
                                 int64_t M_cap, int32_t* offsets, int32_t* token_row,
                                 int32_t* row_token, int32_t* ws, cudaStream_t st);
 // The dispatch in two halves: routing (group offsets, token_row, row_token)
-// and the row copy (pad_only: fill only the rows no pair claimed).
+// and the row copy; for the fused quantize-and-dispatch, the padding rows
+// alone (every row no pair claimed).
 cudaError_t launch_moe_route(const int32_t* topk, int64_t T, int k, int G, int64_t M_cap,
                              int32_t* offsets, int32_t* token_row, int32_t* row_token, int32_t* ws,
                              cudaStream_t st);
 cudaError_t launch_moe_rows(const uint8_t* q, const float* sA, int64_t T, int64_t K,
                             const int32_t* row_token, int64_t M_cap, uint8_t* q_out,
-                            float* sA_out, bool pad_only, cudaStream_t st);
+                            float* sA_out, cudaStream_t st);
+cudaError_t launch_moe_pad_rows(const int32_t* offsets, int G, int64_t K, const int32_t* row_token,
+                                int64_t M_cap, uint8_t* q_out, float* sA_out, cudaStream_t st);
 // 1x128 quantization written straight to the rows token_row gives each token.
 cudaError_t launch_quant_act_1x128_dispatch(const void* x, int in_dtype, int64_t T, int64_t K,
                                             int64_t ldx, const int32_t* token_row, int k,

@@ -158,30 +158,64 @@ __global__ void __launch_bounds__(32) k_moe_rank(const int32_t* __restrict__ top
     }
 }
 
+// A padding row: K zero codes (16-byte stores by the warp's lanes) and K/128
+// scales of 1, what quantizing a zero row gives.
+__device__ __forceinline__ void fill_pad_row(int64_t r, int64_t K, int64_t M_cap, int lane,
+                                             uint8_t* __restrict__ q_out, float* __restrict__ sA_out)
+{
+    uint4* dst = reinterpret_cast<uint4*>(q_out + r * K);
+    for (int64_t v = lane; v < K / 16; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
+    for (int64_t kb = lane; kb < K / 128; kb += 32) sA_out[kb * M_cap + r] = 1.0f;
+}
+
 // CTA = 8 warps, one destination row per warp: the row's K code bytes in
-// 16-byte vectors, then its K/128 scales.  With `pad_only` the rows that hold
-// a pair are left alone (their codes were written by the quantizer itself)
-// and only the padding rows are filled.
+// 16-byte vectors, then its K/128 scales.
 __global__ void __launch_bounds__(256) k_moe_rows(const uint8_t* __restrict__ q,
                                                   const float* __restrict__ sA, int64_t T, int64_t K,
                                                   const int32_t* __restrict__ row_token,
                                                   int64_t M_cap, uint8_t* __restrict__ q_out,
-                                                  float* __restrict__ sA_out, bool pad_only)
+                                                  float* __restrict__ sA_out)
 {
     const int lane = threadIdx.x & 31;
     const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     if (r >= M_cap) return;
     const int32_t t = row_token[r];
-    uint4* dst = reinterpret_cast<uint4*>(q_out + r * K);
-    const int64_t nvec = K / 16;
     if (t >= 0 && t < T) {
-        if (pad_only) return;
+        uint4* dst = reinterpret_cast<uint4*>(q_out + r * K);
         const uint4* src = reinterpret_cast<const uint4*>(q + (int64_t)t * K);
-        for (int64_t v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
+        for (int64_t v = lane; v < K / 16; v += 32) dst[v] = __ldg(src + v);
         for (int64_t kb = lane; kb < K / 128; kb += 32) sA_out[kb * M_cap + r] = __ldg(sA + kb * T + t);
     } else {
-        for (int64_t v = lane; v < nvec; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
-        for (int64_t kb = lane; kb < K / 128; kb += 32) sA_out[kb * M_cap + r] = 1.0f;
+        fill_pad_row(r, K, M_cap, lane, q_out, sA_out);
+    }
+}
+
+// The padding rows only, for the fused quantize-and-dispatch (whose quantizer
+// has written every claimed row).  A group's claimed rows come first, so its
+// padding lies in its last 127 rows; rows from offsets[G] to M_cap are
+// unclaimed.  Warps walk the slots: G x 128 candidate rows (row_token < 0
+// marks padding), then the tail rows; every row written is inside [0, M_cap).
+__global__ void __launch_bounds__(256) k_moe_pad_rows(const int32_t* __restrict__ offsets, int G,
+                                                      int64_t K, const int32_t* __restrict__ row_token,
+                                                      int64_t M_cap, uint8_t* __restrict__ q_out,
+                                                      float* __restrict__ sA_out)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * 8;
+    int64_t end = offsets[G];
+    end = end < 0 ? 0 : (end > M_cap ? M_cap : end);
+    const int64_t slots = (int64_t)G * 128 + (M_cap - end);
+    for (int64_t sl = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); sl < slots; sl += warps) {
+        int64_t r;
+        if (sl < (int64_t)G * 128) {
+            const int e = (int)(sl >> 7);
+            const int64_t lo = offsets[e], hi = offsets[e + 1];
+            r = hi - 128 + (sl & 127);
+            if (r < lo || r < 0 || r >= M_cap || row_token[r] >= 0) continue;
+        } else {
+            r = end + (sl - (int64_t)G * 128);
+        }
+        fill_pad_row(r, K, M_cap, lane, q_out, sA_out);
     }
 }
 
@@ -263,14 +297,25 @@ cudaError_t launch_moe_route(const int32_t* topk, int64_t T, int k, int G, int64
 }
 
 // Row half: copy each claimed row's codes and scales from the token's, and
-// fill the padding rows (or, with pad_only, fill the padding rows only).
+// fill the padding rows.
 cudaError_t launch_moe_rows(const uint8_t* q, const float* sA, int64_t T, int64_t K,
                             const int32_t* row_token, int64_t M_cap, uint8_t* q_out,
-                            float* sA_out, bool pad_only, cudaStream_t st)
+                            float* sA_out, cudaStream_t st)
 {
     if (M_cap > 0)
         k_moe_rows<<<(unsigned)((M_cap + 7) / 8), 256, 0, st>>>(q, sA, T, K, row_token, M_cap,
-                                                              q_out, sA_out, pad_only);
+                                                              q_out, sA_out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_moe_pad_rows(const int32_t* offsets, int G, int64_t K, const int32_t* row_token,
+                                int64_t M_cap, uint8_t* q_out, float* sA_out, cudaStream_t st)
+{
+    if (M_cap <= 0) return cudaSuccess;
+    const int64_t slot_ctas = ((int64_t)G * 128 + M_cap + 7) / 8;
+    const int64_t cap = 4 * (int64_t)device_sm_count();
+    k_moe_pad_rows<<<(unsigned)(slot_ctas < cap ? slot_ctas : cap), 256, 0, st>>>(
+        offsets, G, K, row_token, M_cap, q_out, sA_out);
     return cudaGetLastError();
 }
 
@@ -281,7 +326,7 @@ cudaError_t launch_moe_dispatch(const uint8_t* q, const float* sA, int64_t T, in
 {
     cudaError_t err = launch_moe_route(topk, T, k, G, M_cap, offsets, token_row, row_token, ws, st);
     if (err != cudaSuccess) return err;
-    return launch_moe_rows(q, sA, T, K, row_token, M_cap, q_out, sA_out, false, st);
+    return launch_moe_rows(q, sA, T, K, row_token, M_cap, q_out, sA_out, st);
 }
 
 cudaError_t launch_moe_combine(const void* D, int d_dtype, int64_t M_cap, int64_t N,

@@ -183,8 +183,8 @@ class MoeStep:
     into expert-contiguous, 128-padded FP8 groups (fp8_moe_quant_dispatch)-->,
     W[G,N,K] --128x128-->, grouped GEMM.  `combine(weights)` adds the
     weighted return to token order."""
-    # routing (count, scan, rank), fused quantizer, padding rows, quantize W,
-    # grouped GEMM (+1 memset)
+    # routing (count, scan, rank), fused quantizer, padding rows, quantize W
+    # (on a side stream), grouped GEMM (+1 memset)
     kernel_calls = 7
 
     def __init__(self, x, topk, w, out_dtype=torch.bfloat16, scale_mode=SCALE_FP32,
@@ -210,13 +210,23 @@ class MoeStep:
         self.y = _empty((self.M_cap, N), out_dtype, d)
         self.out = None
         self.inputs, self.output = [x, w, topk], self.y
+        # The weight quantizer has no input in common with the token path, so
+        # it runs on a side stream: the routing kernels (short and latency-
+        # bound) overlap it instead of running alone.
+        self._side = torch.cuda.Stream(device=d)
+        self._fork, self._join = torch.cuda.Event(), torch.cuda.Event()
 
     def quantize(self, stream=None):
-        fp8_moe_quant_dispatch(self.x, self.topk, self.G, self.qa, self.sa, self.offsets,
-                               self.token_row, self.row_token, self.ws, self.mode, stream)
+        cur = stream if stream is not None else torch.cuda.current_stream(self.x.device)
+        self._fork.record(cur)
+        self._side.wait_event(self._fork)
         G, N, K = self.w.shape
         fp8_quant_w_128x128(self.w.view(G * N, K), self.qw.view(G * N, K),
-                            self.sw.view(G * N // 128, K // 128), self.mode, stream)
+                            self.sw.view(G * N // 128, K // 128), self.mode, self._side)
+        fp8_moe_quant_dispatch(self.x, self.topk, self.G, self.qa, self.sa, self.offsets,
+                               self.token_row, self.row_token, self.ws, self.mode, cur)
+        self._join.record(self._side)
+        cur.wait_event(self._join)
 
     def gemm(self, stream=None):
         self._gemm(self.qa, self.sa, self.qw, self.sw, self.offsets, self.y, stream)
