@@ -750,9 +750,8 @@ int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, int b_major
         okB = make_map(&tmB, B, (uint64_t)N, (uint64_t)K, (uint64_t)N, 128, BK);
     }
     if (!okB) return FP8_ERR_LAUNCH;
-    // D as bytes: rows of N * element-size bytes, `ldd` elements apart; the
-    // epilogue stores 32-byte x 32-row boxes
-    // D in its element type; the epilogue stores boxes of 32 bytes x 32 rows
+    // D in its element type, rows `ldd` elements apart; the epilogue stores
+    // boxes of 32 bytes x 32 rows
     CUtensorMap tmD;
     const bool bf16 = out_dtype == FP8_OUT_BF16;
     const uint32_t esz = bf16 ? 2 : 4;

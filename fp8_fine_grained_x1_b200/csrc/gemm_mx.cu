@@ -77,7 +77,10 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_COL0 = BN;
 constexpr uint32_t SF_SLOT_COLS = 16;
 constexpr uint32_t SFB_OFF = 8;
-constexpr int BAND = 16;
+// Raster bands (m-blocks per band): 16 for dense GEMMs; 8 for grouped ones,
+// whose bands otherwise span several experts' rows and weights at once.
+constexpr int BAND_DENSE = 16;
+constexpr int BAND_GROUPED = 8;
 constexpr int SF_AHEAD = 4;                 // K-blocks of scales each writer loads ahead
 constexpr uint32_t SFA_BYTES = 512;              // 128 rows x 4 bytes
 constexpr uint32_t SFB_BYTES = 1024;             // 256 columns x 4 bytes
@@ -100,6 +103,7 @@ struct MxParams {
     int G;
     int b_major, sb_gran, out_dtype;
     int withhold;        // self-test: the odd CTA stops loading after one K-block
+    int band;            // m-blocks per raster band
     uint64_t timeout_ns;
 };
 
@@ -221,7 +225,7 @@ __device__ void mx_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, cons
     mx_unit_range(first, stride);
     for (int64_t tile = first; ok && tile < nmb * nnb; tile += stride) {
         int64_t mb, nb;
-        gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
+        gemm_tile_coord(tile, nmb, nnb, p.band, mb, nb);
         TileRows tr;
         if (!mx_tile_rows(p, sh, mb, rank, tr)) continue;
         const int64_t m0 = tr.m0, n0 = nb * BN;   // an idle odd CTA still loads
@@ -282,7 +286,7 @@ __device__ void mx_mma(const MxParams& p, uint8_t* smem, MxShared& sh, int64_t n
     mx_unit_range(first, stride);
     for (int64_t tile = first; ok && tile < ntiles; tile += stride) {
         int64_t mb, nb;
-        gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
+        gemm_tile_coord(tile, nmb, nnb, p.band, mb, nb);
         const int64_t n0 = nb * BN;
         (void)n0;
         // a pair's MMA always spans 256 columns (a B tail is zero-filled)
@@ -381,7 +385,7 @@ __device__ void mx_scale_writer(const MxParams& p, uint8_t* smem, MxShared& sh, 
     mx_unit_range(first, stride);
     for (int64_t tile = first; ok && tile < nmb * nnb; tile += stride) {
         int64_t mb, nb;
-        gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
+        gemm_tile_coord(tile, nmb, nnb, p.band, mb, nb);
         TileRows tr;
         if (!mx_tile_rows(p, sh, mb, rank, tr)) continue;
         const int64_t n0 = nb * BN;
@@ -438,7 +442,7 @@ __device__ void mx_epilogue(const MxParams& p, MxShared& sh, int64_t nmb, int64_
     mx_unit_range(first, stride);
     for (int64_t tile = first; tile < nmb * nnb; tile += stride) {
         int64_t mb, nb;
-        gemm_tile_coord(tile, nmb, nnb, BAND, mb, nb);
+        gemm_tile_coord(tile, nmb, nnb, p.band, mb, nb);
         TileRows tr;
         if (!mx_tile_rows(p, sh, mb, rank, tr)) continue;
         const uint32_t tph = tcount++ & 1u;
@@ -646,6 +650,7 @@ int launch_mx(const uint8_t* A, const float* sA, const uint8_t* B, int b_major, 
     p.sb_gran = sb_gran;
     p.out_dtype = out_dtype;
     p.withhold = withhold;
+    p.band = group_offsets ? BAND_GROUPED : BAND_DENSE;
     p.timeout_ns = wait_timeout_ns();
 
     const int64_t nnb = (N + BN - 1) / BN;
