@@ -202,8 +202,19 @@ __global__ void __launch_bounds__(256) k_quant_1x128(const Tin* __restrict__ x, 
 // written to every destination row its routing gave it (token_row[t][j],
 // j < k; -1 means the pair was dropped) instead of to the token's own row.
 // The token's codes never round-trip through HBM before the dispatch.
-// Lanes 0..k-1 of each half-warp fetch the token's destinations; a shuffle
-// hands them to the other lanes.  Grid and CTA as k_quant_1x128.
+//
+// A half-warp owns one token and two adjacent K-blocks (256 elements): lane l
+// holds elements 16l .. 16l+15, so lanes 0-7 form the first 1x128 group and
+// lanes 8-15 the second (max-abs over 8 lanes each), and every destination
+// row gets one 16-byte store per lane, 256 contiguous bytes per half-warp.
+// Lanes 0..k-1 fetch the token's destinations; full-warp shuffles (both
+// half-warps walk the same j) hand them to all lanes, and the stores are
+// predicated on the row being valid, so the walk never diverges.
+// CTA = 256 threads = 16 half-warps x 4 tokens each (64 tokens).
+// Grid: x = ceil(K/256) K-block pairs, y = ceil(T/64).
+constexpr int kTokPerHalfWarpDispatch = 4;
+constexpr int kTokPerCtaDispatch = 16 * kTokPerHalfWarpDispatch;   // 64
+
 template <typename Tin>
 __global__ void __launch_bounds__(256) k_quant_1x128_dispatch(
     const Tin* __restrict__ x, int64_t T, int64_t ldx, const int32_t* __restrict__ token_row,
@@ -212,42 +223,52 @@ __global__ void __launch_bounds__(256) k_quant_1x128_dispatch(
 {
     const int h = threadIdx.x >> 4;
     const int l = threadIdx.x & 15;
-    const unsigned half_mask = 0xFFFFu << (threadIdx.x & 16);
-    const int64_t kb = blockIdx.x;
-    const int64_t t0 = (int64_t)blockIdx.y * kRowsPerCta1x128;
+    const int half = threadIdx.x & 16;              // lane offset of this half-warp
+    const int64_t kb = (int64_t)blockIdx.x * 2 + (l >> 3);   // this lane's K-block
+    const bool kb_ok = kb < K / 128;                 // an odd K/128 leaves the last pair half empty
+    const int64_t col = kb * 128 + (l & 7) * 16;     // this lane's first element / code byte
+    const int64_t t0 = (int64_t)blockIdx.y * kTokPerCtaDispatch;
+    uint8_t* const q_col = q_out + col;
+    float* const s_col = sA_out + kb * M_cap;
 
-    Chunk8<Tin> c[kGroupsPerThread1x128];
+    Chunk8<Tin> c[kTokPerHalfWarpDispatch][2];
 #pragma unroll
-    for (int u = 0; u < kGroupsPerThread1x128; ++u) {
+    for (int u = 0; u < kTokPerHalfWarpDispatch; ++u) {
         const int64_t t = t0 + u * 16 + h;
-        if (t < T)
-            c[u].load(x + t * ldx + kb * 128 + l * 8);
-        else
-            c[u].zero();
+        if (t < T && kb_ok) {
+            c[u][0].load(x + t * ldx + col);
+            c[u][1].load(x + t * ldx + col + 8);
+        } else {
+            c[u][0].zero();
+            c[u][1].zero();
+        }
     }
 #pragma unroll
-    for (int u = 0; u < kGroupsPerThread1x128; ++u) {
+    for (int u = 0; u < kTokPerHalfWarpDispatch; ++u) {
         const int64_t t = t0 + u * 16 + h;
-        float v[8];
-        c[u].get(v);
-        float a = absmax8(v);
-        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 8));
+        float v0[8], v1[8];
+        c[u][0].get(v0);
+        c[u][1].get(v1);
+        float a = fmaxf(absmax8(v0), absmax8(v1));
         a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
         a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
         a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
         const GroupScale g = group_scale(a, mode);
-        uint2 out;
-        out.x = encode4(v[0], v[1], v[2], v[3], g.inv);
-        out.y = encode4(v[4], v[5], v[6], v[7], g.inv);
+        uint4 out;
+        out.x = encode4(v0[0], v0[1], v0[2], v0[3], g.inv);
+        out.y = encode4(v0[4], v0[5], v0[6], v0[7], g.inv);
+        out.z = encode4(v1[0], v1[1], v1[2], v1[3], g.inv);
+        out.w = encode4(v1[4], v1[5], v1[6], v1[7], g.inv);
         const bool live = t < T;
         for (int j0 = 0; j0 < k; j0 += 16) {
             const int32_t mine = (live && j0 + l < k) ? __ldg(token_row + t * k + j0 + l) : -1;
             const int nj = k - j0 < 16 ? k - j0 : 16;
             for (int j = 0; j < nj; ++j) {
-                const int32_t r = __shfl_sync(half_mask, mine, j, 16);
-                if (r < 0 || r >= M_cap) continue;
-                *reinterpret_cast<uint2*>(q_out + (int64_t)r * K + kb * 128 + l * 8) = out;
-                if (l == 0) sA_out[kb * M_cap + r] = g.s;
+                const int32_t r = __shfl_sync(0xffffffffu, mine, half + j);
+                if (r >= 0 && r < M_cap && kb_ok) {
+                    *reinterpret_cast<uint4*>(q_col + (int64_t)r * K) = out;
+                    if ((l & 7) == 0) s_col[r] = g.s;
+                }
             }
         }
     }
@@ -654,7 +675,8 @@ cudaError_t launch_quant_act_1x128_dispatch(const void* x, int in_dtype, int64_t
                                             cudaStream_t st)
 {
     if (T == 0) return cudaSuccess;
-    const dim3 grid((unsigned)(K / 128), (unsigned)((T + kRowsPerCta1x128 - 1) / kRowsPerCta1x128));
+    const dim3 grid((unsigned)((K / 128 + 1) / 2),
+                    (unsigned)((T + kTokPerCtaDispatch - 1) / kTokPerCtaDispatch));
     if (in_dtype == FP8_IN_BF16)
         k_quant_1x128_dispatch<__nv_bfloat16><<<grid, 256, 0, st>>>(
             static_cast<const __nv_bfloat16*>(x), T, ldx, token_row, k, M_cap, q_out, K, sA_out,
