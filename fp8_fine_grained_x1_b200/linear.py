@@ -2,7 +2,9 @@
 ready-to-run steps over device-resident inputs.
 
 Each step owns its output buffers (allocated once with torch) and, when
-called, issues only library calls on the current stream:
+called, issues only library calls: on the caller's stream (torch's current
+one by default), and for one of its two quantizers on a side stream forked
+from it and joined back before the GEMM:
 
   FpropStep    X[M,K] --1x128--> (qX, sX);  W[N,K] --128x128--> (qW, sW);
                Y[M,N] = qX . qW^T                      (BF16 or FP32 out)
@@ -43,6 +45,28 @@ def _empty(shape, dtype, device):
     return torch.empty(shape, dtype=dtype, device=device)
 
 
+class _Fork:
+    """Each step's two quantizers share no input, so one of them runs on a
+    side stream forked from the caller's stream and joined back before the
+    GEMM: the tail of one overlaps the other, and short launches overlap
+    each other's start-up."""
+
+    def __init__(self, device):
+        self.side = torch.cuda.Stream(device=device)
+        self.fork, self.join = torch.cuda.Event(), torch.cuda.Event()
+        self.device = device
+
+    def begin(self, stream):
+        cur = stream if stream is not None else torch.cuda.current_stream(self.device)
+        self.fork.record(cur)
+        self.side.wait_event(self.fork)
+        return cur, self.side
+
+    def end(self, cur):
+        self.join.record(self.side)
+        cur.wait_event(self.join)
+
+
 def _gemm_fn(scale_mode, tensor_core_scaling):
     if not tensor_core_scaling:
         return fp8_blockscaled_gemm
@@ -66,10 +90,13 @@ class FpropStep:
         self.y = _empty((M, N), out_dtype, d)
         self.flops = 2 * M * N * K
         self.inputs, self.output = [x, w], self.y
+        self._fork = _Fork(d)
 
     def quantize(self, stream=None):
-        fp8_quant_act_1x128(self.x, self.qx, self.sx, self.mode, stream)
-        fp8_quant_w_128x128(self.w, self.qw, self.sw, self.mode, stream)
+        cur, side = self._fork.begin(stream)
+        fp8_quant_w_128x128(self.w, self.qw, self.sw, self.mode, side)
+        fp8_quant_act_1x128(self.x, self.qx, self.sx, self.mode, cur)
+        self._fork.end(cur)
 
     def gemm(self, stream=None):
         self._gemm(self.qx, self.sx, self.qw, self.sw, self.y, B_KMAJOR, 128, stream)
@@ -98,10 +125,13 @@ class DgradStep:
         self.dx = _empty((M, K_in), out_dtype, d)
         self.flops = 2 * M * K_in * N_out
         self.inputs, self.output = [dy, w], self.dx
+        self._fork = _Fork(d)
 
     def quantize(self, stream=None):
-        fp8_quant_act_1x128(self.dy, self.qdy, self.sdy, self.mode, stream)
-        fp8_quant_w_128x128(self.w, self.qw, self.sw, self.mode, stream)
+        cur, side = self._fork.begin(stream)
+        fp8_quant_w_128x128(self.w, self.qw, self.sw, self.mode, side)
+        fp8_quant_act_1x128(self.dy, self.qdy, self.sdy, self.mode, cur)
+        self._fork.end(cur)
 
     def gemm(self, stream=None):
         # B = W stored [K = N_out][N = K_in]: MN-major; its block scales
@@ -131,10 +161,13 @@ class WgradStep:
         self.dw = _empty((C_out, C_in), torch.float32, d)
         self.flops = 2 * C_out * C_in * T
         self.inputs, self.output = [x, dy], self.dw
+        self._fork = _Fork(d)
 
     def quantize(self, stream=None):
-        fp8_quant_act_128x1(self.dy, self.qdyT, self.sdy, self.mode, stream)
-        fp8_quant_act_128x1(self.x, self.qxT, self.sx, self.mode, stream)
+        cur, side = self._fork.begin(stream)
+        fp8_quant_act_128x1(self.dy, self.qdyT, self.sdy, self.mode, side)
+        fp8_quant_act_128x1(self.x, self.qxT, self.sx, self.mode, cur)
+        self._fork.end(cur)
 
     def gemm(self, stream=None):
         self._gemm(self.qdyT, self.sdy, self.qxT, self.sx, self.dw, B_KMAJOR, 1, stream)
@@ -164,10 +197,13 @@ class WgradCachedStep:
         self.dw = _empty((C_out, C_in), torch.float32, d)
         self.flops = 2 * C_out * C_in * T
         self.inputs, self.output = [qx, sx, dy], self.dw
+        self._fork = _Fork(d)
 
     def quantize(self, stream=None):
-        fp8_quant_act_128x1(self.dy, self.qdyT, self.sdy, self.mode, stream)
-        fp8_requant_1x128_to_128x1(self.qx, self.sx, self.qxT, self.sxT, self.mode, stream)
+        cur, side = self._fork.begin(stream)
+        fp8_quant_act_128x1(self.dy, self.qdyT, self.sdy, self.mode, side)
+        fp8_requant_1x128_to_128x1(self.qx, self.sx, self.qxT, self.sxT, self.mode, cur)
+        self._fork.end(cur)
 
     def gemm(self, stream=None):
         fp8_blockscaled_gemm(self.qdyT, self.sdy, self.qxT, self.sxT, self.dw, B_KMAJOR, 1, stream)
@@ -210,23 +246,18 @@ class MoeStep:
         self.y = _empty((self.M_cap, N), out_dtype, d)
         self.out = None
         self.inputs, self.output = [x, w, topk], self.y
-        # The weight quantizer has no input in common with the token path, so
-        # it runs on a side stream: the routing kernels (short and latency-
-        # bound) overlap it instead of running alone.
-        self._side = torch.cuda.Stream(device=d)
-        self._fork, self._join = torch.cuda.Event(), torch.cuda.Event()
+        # the weight quantizer on the side stream: the short routing kernels
+        # of the token path overlap it
+        self._fork = _Fork(d)
 
     def quantize(self, stream=None):
-        cur = stream if stream is not None else torch.cuda.current_stream(self.x.device)
-        self._fork.record(cur)
-        self._side.wait_event(self._fork)
+        cur, side = self._fork.begin(stream)
         G, N, K = self.w.shape
         fp8_quant_w_128x128(self.w.view(G * N, K), self.qw.view(G * N, K),
-                            self.sw.view(G * N // 128, K // 128), self.mode, self._side)
+                            self.sw.view(G * N // 128, K // 128), self.mode, side)
         fp8_moe_quant_dispatch(self.x, self.topk, self.G, self.qa, self.sa, self.offsets,
                                self.token_row, self.row_token, self.ws, self.mode, cur)
-        self._join.record(self._side)
-        cur.wait_event(self._join)
+        self._fork.end(cur)
 
     def gemm(self, stream=None):
         self._gemm(self.qa, self.sa, self.qw, self.sw, self.offsets, self.y, stream)
