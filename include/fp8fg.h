@@ -270,7 +270,7 @@ int fp8_moe_dispatch(const uint8_t* q, const float* sA, int64_t T, int64_t K, co
  *   the other arguments as fp8_moe_dispatch (same workspace size)
  * Sizes: as fp8_moe_dispatch, plus ldx >= K and ldx * element size a
  * multiple of 16 bytes; x 16-byte aligned.  Errors as fp8_moe_dispatch.
- * Launches four kernels and one memset: the routing passes, the fused
+ * Launches five kernels and one memset: three routing passes, the fused
  * quantizer, and a pass that fills the padding rows.
  */
 int fp8_moe_quant_dispatch(const void* x, int in_dtype, int64_t T, int64_t K, int64_t ldx,

@@ -130,6 +130,25 @@ def test_quant_dispatch_reports_bad_expert_ids_like_the_dispatch():
     assert torch.equal(got["sA"].view(torch.int32), ref["sA"].view(torch.int32))
 
 
+@pytest.mark.parametrize("M_cap", [384, 640])
+def test_quant_dispatch_over_capacity_matches_the_dispatch(M_cap):
+    """A capacity below the padded total: both paths report it, drop the same
+    pairs, and write the same rows (the padding kernel of the fused path only
+    visits each group's last 127 rows and the unclaimed tail)."""
+    T, K, k, G = 200, 256, 3, 5
+    x = synth.activations(T, K, seed=41, outlier_seed=42).to(dev())
+    topk = synth.zipf_topk_routing(T, G, k, seed=43).numpy().astype(np.int32)
+    got = _quant_dispatch(x, topk, G, fg.SCALE_FP32, M_cap=M_cap)
+    assert fg.fp8_get_status() == fg.FP8_ERR_SHAPE
+    qx, sx = fg.quant_act_1x128(x)
+    ref = fg.moe_dispatch(qx, sx, to_dev(topk), G, M_cap=M_cap)
+    assert fg.fp8_get_status() == fg.FP8_ERR_SHAPE
+    for key in ("offsets", "token_row", "row_token", "q"):
+        assert torch.equal(got[key], ref[key]), key
+    assert torch.equal(got["sA"].view(torch.int32), ref["sA"].view(torch.int32))
+    assert fg.fp8_get_status() == fg.FP8_OK
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
 def test_combine_matches_oracle(dtype):
     rng = np.random.default_rng(3)
