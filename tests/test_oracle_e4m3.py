@@ -120,13 +120,17 @@ def test_encode_zero_and_underflow_keep_sign():
 
 
 @pytest.mark.slow
-def test_encode_dense_sweep_against_library():
-    """Every 7th FP32 bit pattern of [0, 448] (about 1.6e8 values) in chunks."""
+def test_encode_exhaustive_against_library():
+    """Every FP32 bit pattern of [0, 448] (about 1.14e9 values), in chunks,
+    against the library cast; the negative patterns follow by the sign bit
+    (checked on a strided sample here and in the tests above)."""
     hi_bits = int(np.float32(448.0).view(np.uint32))
-    step = 7
     for start in range(0, hi_bits + 1, 1 << 26):
-        b = np.arange(start, min(start + (1 << 26), hi_bits + 1), step, dtype=np.uint32)
+        b = np.arange(start, min(start + (1 << 26), hi_bits + 1), dtype=np.uint32)
         v = b.view(np.float32)
         ours = oracle.e4m3_encode_array(v)
         lib = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
-        assert np.array_equal(ours, lib)
+        assert np.array_equal(ours, lib), start
+    neg = -np.arange(0, hi_bits + 1, 9973, dtype=np.uint32).view(np.float32)
+    assert np.array_equal(oracle.e4m3_encode_array(neg),
+                          torch.from_numpy(neg).to(torch.float8_e4m3fn).view(torch.uint8).numpy())
