@@ -142,3 +142,35 @@ def test_full_size_wgrad_operands_bitexact(mode):
         torch.cuda.synchronize()
         assert np.array_equal(q.cpu().numpy(), q_ref)
         assert np.array_equal(s.cpu().numpy(), s_ref)
+
+
+def test_gpu_encode_of_every_fp32_pattern_in_range():
+    """The GPU's E4M3 encode on every FP32 bit pattern of [0, 448]: each 1x128
+    group holds 448 in its first lane, so its scale is amax/448 = 1 and its
+    encode factor 448/amax = 1, and every other lane's code is E(x) of its
+    own value.  Compared with the oracle's encoder (itself pinned to the
+    library cast on the same patterns); negatives on a strided sample."""
+    hi_bits = int(np.float32(448.0).view(np.uint32))
+    per = 127 << 19                                     # values per launch, 127 per group
+    for start in range(0, hi_bits + 1, per):
+        b = np.arange(start, min(start + per, hi_bits + 1), dtype=np.uint32)
+        _encode_groups_match(b.view(np.float32))
+    neg = -np.arange(0, hi_bits + 1, 9973, dtype=np.uint32).view(np.float32)
+    _encode_groups_match(neg)
+
+
+def _encode_groups_match(vals):
+    n = vals.size
+    G = (n + 126) // 127
+    body = np.zeros(G * 127, np.float32)
+    body[:n] = vals
+    x = np.empty((G, 128), np.float32)
+    x[:, 0] = 448.0
+    x[:, 1:] = body.reshape(G, 127)
+    q, s = fg.quant_act_1x128(to_dev(x))
+    assert fg.fp8_get_status() == fg.FP8_OK
+    assert torch.all(s == 1.0).item()
+    got = q[:, 1:].reshape(-1)[:n].cpu().numpy()
+    ref = oracle.e4m3_encode_array(vals)
+    bad = np.flatnonzero(got != ref)
+    assert bad.size == 0, (vals[bad[:8]], got[bad[:8]], ref[bad[:8]])
