@@ -174,3 +174,22 @@ def _encode_groups_match(vals):
     ref = oracle.e4m3_encode_array(vals)
     bad = np.flatnonzero(got != ref)
     assert bad.size == 0, (vals[bad[:8]], got[bad[:8]], ref[bad[:8]])
+
+
+@pytest.mark.parametrize("mode", [fg.SCALE_FP32, fg.SCALE_POW2])
+def test_gpu_group_scale_across_the_fp32_range(mode):
+    """Group scales for maxima spread over every binade of FP32 (every 4096th
+    bit pattern from the smallest subnormal to the largest finite value, and
+    their negatives): one nonzero element per 1x128 group, scale and codes
+    bit-exact against the oracle."""
+    top = int(np.float32(np.finfo(np.float32).max).view(np.uint32))
+    v = np.arange(1, top + 1, 4096, dtype=np.uint32).view(np.float32)
+    v = np.concatenate([v, -v[::7]])
+    x = np.zeros((v.size, 128), np.float32)
+    lanes = np.arange(v.size) % 128                      # the nonzero element visits every lane
+    x[np.arange(v.size), lanes] = v
+    q, s = fg.quant_act_1x128(to_dev(x), mode)
+    assert fg.fp8_get_status() == fg.FP8_OK
+    oq, os_ = oracle.quant_act_1x128(x, mode)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), os_.view(np.uint32))
+    assert np.array_equal(q.cpu().numpy(), oq)
