@@ -82,10 +82,10 @@ static_assert(128 * CTRL_REGS + 256 * PROMO_REGS <= NUM_THREADS * LAUNCH_REGS,
 constexpr int PROMO_CHUNK = 32;                        // TMEM columns per load round trip
 constexpr uint32_t TMEM_COLS = 2 * BN;                  // two FP32 partial buffers
 constexpr int MAX_GROUPS = 1024;
-// Raster bands (m-blocks per band): 16 for dense GEMMs; 8 for grouped ones,
+// Raster bands (m-blocks per band): 16 for dense GEMMs; 6 for grouped ones,
 // whose bands otherwise span several experts' rows and weights at once.
 constexpr int BAND_DENSE = 16;
-constexpr int BAND_GROUPED = 8;
+constexpr int BAND_GROUPED = 6;
 constexpr uint32_t DYN_SMEM = 1024 + RING_BYTES;
 
 struct GemmParams {
