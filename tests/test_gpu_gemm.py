@@ -149,6 +149,28 @@ def test_grouped_matches_oracle(counts, N, K, out):
     assert np.all(got[pad] == 0.0)
 
 
+@pytest.mark.parametrize("out", ["bf16", "fp32"])
+def test_grouped_many_groups_across_raster_bands(out):
+    """40 experts of 0..700 rows (odd and even 128-row block counts, empty
+    ones): the 256-row pair blocks span several raster bands and N-blocks,
+    so band boundaries fall inside and between groups.  Full output."""
+    rng = np.random.default_rng(91)
+    counts = [int(c) for c in rng.integers(0, 700, 40)]
+    counts[3] = counts[17] = 0
+    N, K = 512, 256
+    A, sA, B, sB, off = _grouped_operands(counts, N, K, seed=900)
+    dt = torch.bfloat16 if out == "bf16" else torch.float32
+    D = torch.full((A.shape[0], N), -3.0, dtype=dt, device=dev())
+    fg.fp8_grouped_gemm(to_dev(A), to_dev(sA), to_dev(B), to_dev(sB), to_dev(off), D)
+    assert fg.fp8_get_status() == fg.FP8_OK
+    got = d2h(D)
+    mm, nn = np.meshgrid(np.arange(A.shape[0]), np.arange(N), indexing="ij")
+    pts = np.stack([mm.reshape(-1), nn.reshape(-1)], axis=1).astype(np.int64)
+    ref, tol, grp = oracle.grouped_gemm_points(A, sA, B, sB, off, pts)
+    assert np.all(grp >= 0)
+    assert_gemm_close(got.reshape(-1), ref, tol, out == "bf16", "grouped, many groups")
+
+
 def test_grouped_bad_offsets_report_shape_error_and_write_nothing():
     N, K = 256, 256
     A, sA, B, sB, off = _grouped_operands([128, 128], N, K, seed=5)
