@@ -18,6 +18,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 
 #include "fp8fg_device.cuh"
 #include "fp8fg_host.h"
@@ -519,9 +520,10 @@ __global__ void __launch_bounds__(kThr128x1, 5) k_quant_128x1(const Tin* __restr
 // max-abs, combined over the 8 warps through shared memory, where thread c
 // (c < 128) derives channel c's scale once for the CTA.  Pass 2: each
 // thread encodes its 16 tokens of each of its 4 channels into one 16-byte
-// word.  The staged tile is dead by then, so the transposed codes go
-// back into the same buffer (16-byte chunks XOR-swizzled by (channel / 4) %
-// 8, conflict-free) and leave as coalesced 128-byte rows of qT.
+// word.  The transposed codes go into their own buffer (16-byte chunks
+// XOR-swizzled by (channel / 4) % 8, conflict-free) and leave as coalesced
+// 128-byte rows of qT; with the staged codes in separate buffers, a tile
+// needs four block barriers, none at its end.
 // Grid: x = C/128, y = ceil(T/128 / kReqTiles).
 constexpr int kReqTok = 128;
 constexpr int kReqCh = 128;
@@ -545,15 +547,26 @@ __device__ __forceinline__ void decode4_e4m3(uint32_t w, float (&f)[4])
         : "r"(w));
 }
 
+struct __align__(16) ReqShared {
+    uint8_t tile[2][kReqTok * kReqCh];   // staged codes, double-buffered
+    uint8_t outT[kReqCh * kReqTok];      // the current tile's transposed codes
+    float part[8][kReqCh];               // per-warp max-abs of each channel
+    float inv_s[kReqCh];                 // per-channel encode factors of the tile
+    float scl[2][kReqTok];               // staged 1x128 scales of the tile's tokens
+};
+constexpr uint32_t kReqSmemBytes = (uint32_t)sizeof(ReqShared);
+
 __global__ void __launch_bounds__(256, 3) k_requant_128x1(const uint8_t* __restrict__ q, int64_t ldq,
                                                        const float* __restrict__ sA, int64_t T,
                                                        int64_t C, uint8_t* __restrict__ qT,
                                                        int64_t ldqT, float* __restrict__ s, int mode)
 {
-    __shared__ __align__(16) uint8_t tile[2][kReqTok * kReqCh];   // codes, then transposed codes
-    __shared__ __align__(16) float part[8][kReqCh];
-    __shared__ __align__(16) float inv_s[kReqCh];   // per-channel encode factors of the tile
-    __shared__ __align__(16) float scl[2][kReqTok];
+    extern __shared__ __align__(16) uint8_t req_raw[];
+    ReqShared& sh = *reinterpret_cast<ReqShared*>(req_raw);
+    auto& tile = sh.tile;
+    auto& part = sh.part;
+    auto& inv_s = sh.inv_s;
+    auto& scl = sh.scl;
 
     const int64_t cb = blockIdx.x;
     const int64_t c0 = cb * kReqCh;
@@ -617,7 +630,7 @@ __global__ void __launch_bounds__(256, 3) k_requant_128x1(const uint8_t* __restr
             inv_s[c] = gs.inv;
             s[tb * C + c0 + c] = gs.s;
         }
-        __syncthreads();   // inv_s is ready; every read of the staged codes is done
+        __syncthreads();   // inv_s is ready
         const float4 inv4 = *reinterpret_cast<const float4*>(&inv_s[4 * lane]);
         const float inv[4] = {inv4.x, inv4.y, inv4.z, inv4.w};
 
@@ -630,7 +643,7 @@ __global__ void __launch_bounds__(256, 3) k_requant_128x1(const uint8_t* __restr
                 out[k][q4] = encode4(v[4 * q4][k], v[4 * q4 + 1][k], v[4 * q4 + 2][k], v[4 * q4 + 3][k],
                                      inv[k]);
         }
-        uint8_t* tl = tile[buf];
+        uint8_t* tl = sh.outT;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const int c = 4 * lane + k;
@@ -647,7 +660,11 @@ __global__ void __launch_bounds__(256, 3) k_requant_128x1(const uint8_t* __restr
             const uint4 v = *reinterpret_cast<const uint4*>(&tl[c * kReqTok + ((chunk ^ ((c >> 2) & 7)) * 16)]);
             *reinterpret_cast<uint4*>(qT + (c0 + c) * ldqT + t0 + chunk * 16) = v;
         }
-        __syncthreads();   // this buffer may be refilled by the next prefetch
+        // No barrier here.  The next tile's prefetch into this tile's staging
+        // buffer comes after this tile's second barrier, which follows every
+        // thread's reads of the staged codes and scales; the next tile's
+        // writes of part, inv_s and outT come after the next tile's first
+        // barrier, which every thread passes only after finishing this tile.
     }
     cp_async_wait_group<0>();
 }
@@ -708,9 +725,22 @@ cudaError_t launch_requant_128x1(const uint8_t* q, int64_t ldq, const float* sA,
                                  int64_t C, uint8_t* qT, int64_t ldqT, float* s, int mode,
                                  cudaStream_t st)
 {
+    static bool ready[64] = {};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (!ready[dev]) {   // above the 48 KB default for dynamic shared memory
+            const cudaError_t e = cudaFuncSetAttribute(
+                k_requant_128x1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kReqSmemBytes);
+            if (e != cudaSuccess) return e;
+            ready[dev] = true;
+        }
+    }
     const int64_t ntb = T / kReqTok;
     const dim3 grid((unsigned)(C / kReqCh), (unsigned)((ntb + kReqTiles - 1) / kReqTiles));
-    k_requant_128x1<<<grid, 256, 0, st>>>(q, ldq, sA, T, C, qT, ldqT, s, mode);
+    k_requant_128x1<<<grid, 256, kReqSmemBytes, st>>>(q, ldq, sA, T, C, qT, ldqT, s, mode);
     return cudaGetLastError();
 }
 
