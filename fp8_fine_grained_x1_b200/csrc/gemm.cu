@@ -303,6 +303,9 @@ __device__ void run_mma(const GemmParams& p, uint8_t* smem, Shared& sh, int64_t 
     mbar_wait_drain(&sh.drain, 0, p.timeout_ns);
 }
 
+// GRAN is the weight-scale granularity along N (p.sb_gran): 128 (one scale
+// per 128x128 block) or 1 (one per column); each gets its own instance.
+template <int GRAN>
 __device__ void run_promotion(const CUtensorMap* tmD, const GemmParams& p, Shared& sh, int nmb,
                               int nnb, int nkb, int warp, int lane)
 {
@@ -344,10 +347,10 @@ __device__ void run_promotion(const CUtensorMap* tmD, const GemmParams& p, Share
         //        warp's shared buffer so every lane can read all 128.
         const float* sa_ptr = p.sA + (row_ok ? m + (int64_t)kb0 * p.M : 0);
         const int64_t sa_step = row_ok ? p.M : 0;
-        const bool use_sb = active && p.sb_gran == 128;
+        const bool use_sb = active && GRAN == 128;
         const float* sb_ptr = p.sB;
         int64_t sb_step = 0;
-        if (p.sb_gran == 128) {
+        if (GRAN == 128) {
             if (p.b_major == FP8_B_KMAJOR) {
                 sb_ptr = p.sB + ((int64_t)g * nnb128 + cb) * nkb + kb0;
                 sb_step = 1;
@@ -356,7 +359,7 @@ __device__ void run_promotion(const CUtensorMap* tmD, const GemmParams& p, Share
                 sb_step = nnb128;
             }
         }
-        const bool use_sb4 = active && p.sb_gran == 1;
+        const bool use_sb4 = active && GRAN == 1;
         const float4* sb4_ptr =
             reinterpret_cast<const float4*>(p.sB + (int64_t)kb0 * p.N + n0 + col0) + lane;
         const int64_t sb4_step = p.N / 4;
@@ -367,7 +370,7 @@ __device__ void run_promotion(const CUtensorMap* tmD, const GemmParams& p, Share
 
         float sa_next = row_ok ? __ldg(sa_ptr) : 0.0f;
         float sb_next = use_sb ? __ldg(sb_ptr) : 0.0f;
-        if (p.sb_gran == 1) {
+        if (GRAN == 1) {
             *reinterpret_cast<float4*>(&sh.sbw[ew][kb0 & 1][lane * 4]) =
                 use_sb4 ? __ldg(sb4_ptr) : make_float4(0.f, 0.f, 0.f, 0.f);
             __syncwarp();
@@ -396,7 +399,7 @@ __device__ void run_promotion(const CUtensorMap* tmD, const GemmParams& p, Share
                 // PROMO_CHUNK columns per TMEM round trip: their 16-column
                 // loads are all in flight before the first wait.
                 constexpr int NL = PROMO_CHUNK / 16;
-                if (p.sb_gran == 128) {
+                if (GRAN == 128) {
                     const float sc = sa * sb;
 #pragma unroll
                     for (int c = 0; c < 128 / PROMO_CHUNK; ++c) {
@@ -415,27 +418,32 @@ __device__ void run_promotion(const CUtensorMap* tmD, const GemmParams& p, Share
                             }
                     }
                 } else {
+                    // The chunk's products sa * sb[col] only need shared memory
+                    // and registers, so they are formed while its TMEM loads
+                    // are in flight; after the wait only the FMAs remain.
                     const float* sbv = sh.sbw[ew][kb & 1];
 #pragma unroll
                     for (int c = 0; c < 128 / PROMO_CHUNK; ++c) {
                         uint32_t r[NL][16];
 #pragma unroll
                         for (int l = 0; l < NL; ++l) tmem_ld16(taddr + c * PROMO_CHUNK + l * 16, r[l]);
+                        float t[PROMO_CHUNK];
+#pragma unroll
+                        for (int i = 0; i < PROMO_CHUNK / 4; ++i) {
+                            const float4 b = *reinterpret_cast<const float4*>(sbv + c * PROMO_CHUNK + 4 * i);
+                            fmul2(t[4 * i], t[4 * i + 1], b.x, b.y, sa, sa);
+                            fmul2(t[4 * i + 2], t[4 * i + 3], b.z, b.w, sa, sa);
+                        }
 #pragma unroll
                         for (int l = 0; l < NL; ++l) tmem_ld_wait(r[l]);
 #pragma unroll
                         for (int l = 0; l < NL; ++l)
 #pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const int j = c * PROMO_CHUNK + l * 16 + 4 * i;
-                                const float4 b = *reinterpret_cast<const float4*>(sbv + j);
-                                float t0, t1, t2, t3;
-                                fmul2(t0, t1, b.x, b.y, sa, sa);
-                                fmul2(t2, t3, b.z, b.w, sa, sa);
-                                ffma2(acc[j], acc[j + 1], __uint_as_float(r[l][4 * i]),
-                                      __uint_as_float(r[l][4 * i + 1]), t0, t1);
-                                ffma2(acc[j + 2], acc[j + 3], __uint_as_float(r[l][4 * i + 2]),
-                                      __uint_as_float(r[l][4 * i + 3]), t2, t3);
+                            for (int i = 0; i < 8; ++i) {
+                                const int j = c * PROMO_CHUNK + l * 16 + 2 * i;
+                                ffma2(acc[j], acc[j + 1], __uint_as_float(r[l][2 * i]),
+                                      __uint_as_float(r[l][2 * i + 1]), t[l * 16 + 2 * i],
+                                      t[l * 16 + 2 * i + 1]);
                             }
                     }
                 }
@@ -444,7 +452,7 @@ __device__ void run_promotion(const CUtensorMap* tmD, const GemmParams& p, Share
             __syncwarp();
             // the even CTA's MMA waits for both CTAs' warps
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&sh.tempty[buf]), 0));
-            if (p.sb_gran == 1) {
+            if (GRAN == 1) {
                 *reinterpret_cast<float4*>(&sh.sbw[ew][(kb + 1) & 1][lane * 4]) = sb4_next;
                 __syncwarp();
             }
@@ -575,7 +583,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     } else {
         regs_inc<PROMO_REGS>();
-        if (!sh.bad) run_promotion(&tmD, p, sh, (int)nmb, (int)nnb, (int)nkb, warp, lane);
+        if (!sh.bad) {
+            if (p.sb_gran == 128)
+                run_promotion<128>(&tmD, p, sh, (int)nmb, (int)nnb, (int)nkb, warp, lane);
+            else
+                run_promotion<1>(&tmD, p, sh, (int)nmb, (int)nnb, (int)nkb, warp, lane);
+        }
     }
     tc_fence_before();
     cluster_sync();
