@@ -400,22 +400,36 @@ __device__ void run_promotion(const CUtensorMap* tmD, const GemmParams& p, Share
                 // loads are all in flight before the first wait.
                 constexpr int NL = PROMO_CHUNK / 16;
                 if (GRAN == 128) {
+                    // the next chunk's loads are in flight while this chunk's
+                    // FMAs run (two register sets, used in turn)
                     const float sc = sa * sb;
+                    constexpr int NC = 128 / PROMO_CHUNK;
+                    uint32_t ra[NL][16], rb[NL][16];
 #pragma unroll
-                    for (int c = 0; c < 128 / PROMO_CHUNK; ++c) {
-                        uint32_t r[NL][16];
+                    for (int l = 0; l < NL; ++l) tmem_ld16(taddr + l * 16, ra[l]);
 #pragma unroll
-                        for (int l = 0; l < NL; ++l) tmem_ld16(taddr + c * PROMO_CHUNK + l * 16, r[l]);
+                    for (int l = 0; l < NL; ++l) tmem_ld_wait(ra[l]);
 #pragma unroll
-                        for (int l = 0; l < NL; ++l) tmem_ld_wait(r[l]);
+                    for (int c = 0; c < NC; ++c) {
+                        uint32_t (&cur)[NL][16] = (c & 1) ? rb : ra;
+                        uint32_t (&nxt)[NL][16] = (c & 1) ? ra : rb;
+                        if (c + 1 < NC) {
+#pragma unroll
+                            for (int l = 0; l < NL; ++l)
+                                tmem_ld16(taddr + (c + 1) * PROMO_CHUNK + l * 16, nxt[l]);
+                        }
 #pragma unroll
                         for (int l = 0; l < NL; ++l)
 #pragma unroll
                             for (int i = 0; i < 8; ++i) {
                                 const int j = c * PROMO_CHUNK + l * 16 + 2 * i;
-                                ffma2(acc[j], acc[j + 1], __uint_as_float(r[l][2 * i]),
-                                      __uint_as_float(r[l][2 * i + 1]), sc, sc);
+                                ffma2(acc[j], acc[j + 1], __uint_as_float(cur[l][2 * i]),
+                                      __uint_as_float(cur[l][2 * i + 1]), sc, sc);
                             }
+                        if (c + 1 < NC) {
+#pragma unroll
+                            for (int l = 0; l < NL; ++l) tmem_ld_wait(nxt[l]);
+                        }
                     }
                 } else {
                     // The chunk's products sa * sb[col] only need shared memory
