@@ -47,6 +47,7 @@ EXPORTED = (
     "fp8_moe_dispatch_workspace_bytes", "fp8_moe_dispatch", "fp8_moe_combine",
     "fp8_moe_dispatch_noalloc", "fp8_requant_1x128_to_128x1", "fp8_blockscaled_gemm_pow2",
     "fp8_grouped_gemm_pow2", "fp8_moe_quant_dispatch", "fp8_selftest_gemm_unwind",
+    "fp8_grouped_gemm_gather", "fp8_moe_route",
 )
 
 
@@ -84,6 +85,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fp8_grouped_gemm_pow2.restype = _I
     lib.fp8_grouped_gemm.argtypes = [_P, _P, _P, _P, _P, _I, _I64, _I64, _I64, _P, _I, _P]
     lib.fp8_grouped_gemm.restype = _I
+    lib.fp8_grouped_gemm_gather.argtypes = [_P, _P, _I64, _P, _P, _P, _P, _I, _I64, _I64, _I64, _P,
+                                            _I, _P]
+    lib.fp8_grouped_gemm_gather.restype = _I
+    lib.fp8_moe_route.argtypes = [_P, _I64, _I, _I, _I64, _P, _P, _P, _P, _I64, _P]
+    lib.fp8_moe_route.restype = _I
     lib.fp8_get_status.argtypes = [_P]
     lib.fp8_get_status.restype = _I
     lib.fp8_status_string.argtypes = [_I]
@@ -231,6 +237,27 @@ def fp8_grouped_gemm(A, sA, B, sB, group_offsets, D, stream=None) -> None:
     _check(load_library().fp8_grouped_gemm(
         _ptr(A), _ptr(sA), _ptr(B), _ptr(sB), _ptr(group_offsets), G, M_total, N, K, _ptr(D),
         _out_dtype(D), _stream(stream)), "fp8_grouped_gemm")
+
+
+def fp8_grouped_gemm_gather(A, sA, row_token, B, sB, group_offsets, D, stream=None) -> None:
+    """Output row m of D [M_total, N] = token row row_token[m] of A [T, K]
+    (sA [K/128, T]) times its expert's weight (B [G, N, K]); -1 rows give 0."""
+    T, K = A.shape
+    G, N, _ = B.shape
+    M_total = D.shape[0]
+    _check(load_library().fp8_grouped_gemm_gather(
+        _ptr(A), _ptr(sA), T, _ptr(row_token), _ptr(B), _ptr(sB), _ptr(group_offsets), G, M_total,
+        N, K, _ptr(D), _out_dtype(D), _stream(stream)), "fp8_grouped_gemm_gather")
+
+
+def fp8_moe_route(topk, G, group_offsets, token_row, row_token, workspace, stream=None) -> None:
+    """The routing of fp8_moe_dispatch alone (offsets, token_row, row_token)."""
+    T, k = topk.shape
+    M_cap = row_token.shape[0]
+    _check(load_library().fp8_moe_route(
+        _ptr(topk), T, k, G, M_cap, _ptr(group_offsets), _ptr(token_row), _ptr(row_token),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
+        "fp8_moe_route")
 
 
 def fp8_moe_dispatch_workspace_bytes(T: int, k: int, G: int) -> int:

@@ -220,6 +220,49 @@ FP8FG_API int fp8_grouped_gemm(const uint8_t* A, const float* sA, const uint8_t*
                                    D, out_dtype, N, static_cast<cudaStream_t>(stream));
 }
 
+FP8FG_API int fp8_grouped_gemm_gather(const uint8_t* A, const float* sA, int64_t T,
+                                      const int32_t* row_token, const uint8_t* B, const float* sB,
+                                      const int32_t* group_offsets, int G, int64_t M_total,
+                                      int64_t N, int64_t K, void* D, int out_dtype, void* stream)
+{
+    if (!is_out(out_dtype)) return FP8_ERR_DTYPE;
+    if (G < 1 || G > 1024 || M_total < 0 || M_total > kMaxDim || M_total % 128 || N <= 0 ||
+        N > kMaxDim || N % 128 || K <= 0 || K > kMaxDim || K % 128 || (int64_t)G * N > kMaxDim ||
+        T < 0 || T > kMaxDim)
+        return FP8_ERR_SHAPE;
+    if (M_total == 0) return FP8_OK;
+    if (T < 1) return FP8_ERR_SHAPE;   // every row of D would be padding
+    if (!A || !sA || !row_token || !B || !sB || !group_offsets || !D) return FP8_ERR_NULL;
+    const int osz = out_dtype == FP8_OUT_BF16 ? 2 : 4;
+    if (!aligned(A, 16) || !aligned(B, 16) || !aligned(D, 16) || !aligned(sA, 4) ||
+        !aligned(sB, 4) || !aligned(group_offsets, 4) || !aligned(row_token, 4) || (N * osz) % 16)
+        return FP8_ERR_ALIGN;
+    if (!device_is_sm100()) return FP8_ERR_DEVICE;
+    return launch_grouped_gemm_gather(A, sA, T, row_token, B, sB, group_offsets, G, M_total, N, K, D,
+                                      out_dtype, static_cast<cudaStream_t>(stream));
+}
+
+FP8FG_API int fp8_moe_route(const int32_t* topk, int64_t T, int k, int G, int64_t M_cap,
+                            int32_t* group_offsets, int32_t* token_row, int32_t* row_token,
+                            void* workspace, int64_t workspace_bytes, void* stream)
+{
+    if (T < 0 || k < 1 || G < 1 || G > 1024 || M_cap < 0 || M_cap % 128 || M_cap > kMaxDim ||
+        T > kMaxPairs / k)
+        return FP8_ERR_SHAPE;
+    if (workspace_bytes < fp8_moe_dispatch_workspace_bytes(T, k, G)) return FP8_ERR_SHAPE;
+    if (!group_offsets || (T > 0 && (!topk || !token_row || !workspace)) || (M_cap > 0 && !row_token))
+        return FP8_ERR_NULL;
+    if (!aligned(topk, 4) || !aligned(group_offsets, 4) || !aligned(token_row, 4) ||
+        !aligned(row_token, 4) || !aligned(workspace, 4))
+        return FP8_ERR_ALIGN;
+    if (!device_is_sm100()) return FP8_ERR_DEVICE;
+    return launch_moe_route(topk, T, k, G, M_cap, group_offsets, token_row, row_token,
+                            static_cast<int32_t*>(workspace), static_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? FP8_OK
+               : FP8_ERR_LAUNCH;
+}
+
 FP8FG_API int64_t fp8_moe_dispatch_workspace_bytes(int64_t T, int k, int G)
 {
     if (T < 0 || k < 1 || G < 1 || G > 1024 || T > kMaxPairs / k) return 0;

@@ -275,6 +275,23 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorM
         : "memory");
 }
 
+// TMA 2-D gather of four whole rows (row indices r0..r3, columns from x on,
+// one box of the tensor map per row; the map's box is one row high) into
+// consecutive rows of this CTA's shared memory, with the same 128-byte
+// swizzle a tiled load of those rows would give.  Bytes count on an mbarrier
+// of either CTA of the pair.  No cluster multicast.
+__device__ __forceinline__ void tma_gather4_pair(void* smem_dst, const CUtensorMap* map,
+                                                 uint32_t bar_cluster_addr, int32_t x, int32_t r0,
+                                                 int32_t r1, int32_t r2, int32_t r3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(x), "r"(r0), "r"(r1), "r"(r2),
+        "r"(r3)
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* smem_dst, uint32_t ncols)
 {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(

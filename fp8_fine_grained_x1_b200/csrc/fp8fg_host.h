@@ -27,6 +27,12 @@ int launch_blockscaled_gemm(const uint8_t* A, const float* sA, const uint8_t* B,
                             const float* sB, int sb_gran, int64_t M, int64_t N, int64_t K,
                             const int32_t* group_offsets, int G, void* D, int out_dtype,
                             int64_t ldd, cudaStream_t st);
+// Grouped GEMM whose A rows are gathered: output row m reads A row row_map[m]
+// of A [a_rows][K] (sA [K/128][a_rows]); -1 marks a padding row (output 0).
+int launch_grouped_gemm_gather(const uint8_t* A, const float* sA, int64_t a_rows,
+                               const int32_t* row_map, const uint8_t* B, const float* sB,
+                               const int32_t* group_offsets, int G, int64_t M, int64_t N, int64_t K,
+                               void* D, int out_dtype, cudaStream_t st);
 
 // Self-test forms of the two GEMMs: the odd CTA of every pair withholds its
 // operand loads after its first K-block, so the pair's waits run out.

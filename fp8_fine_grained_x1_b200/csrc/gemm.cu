@@ -99,6 +99,8 @@ struct GemmParams {
     int band;                      // m-blocks per raster band
     int streamk;                   // 1: contiguous ranges of (tile, K-block) units per pair
     int withhold;                  // self-test: the odd CTA stops loading after one K-block
+    const int32_t* row_map;        // grouped gather: A row of each output row (nullptr: A as is)
+    int64_t a_rows;                // gather: rows of A (and of sA's K-block rows)
     uint64_t timeout_ns;
 };
 
@@ -201,8 +203,13 @@ __device__ __forceinline__ void seg_next(Segments& g)
     }
 }
 
+// Run by the whole of warp 0.  Lane 0 arms the stage barrier and issues the
+// tiled loads; with gathered A each lane issues one 4-row gather (rows
+// 4*lane .. 4*lane+3 of the CTA's 128), so a stage's 32 gathers leave in one
+// warp instruction.  Every decision is warp-uniform.
 __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, const GemmParams& p,
-                             uint8_t* smem, Shared& sh, int64_t nmb, int64_t nnb, int64_t nkb)
+                             uint8_t* smem, Shared& sh, int64_t nmb, int64_t nnb, int64_t nkb,
+                             int lane)
 {
     volatile int* abort = &sh.abort;
     const uint32_t rank = cluster_ctarank();
@@ -221,6 +228,18 @@ __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, con
         // A CTA of a pair loads B's columns rank*128 .. rank*128+127 of the
         // tile (a box counts in full, its out-of-range part zero-filled).
         const int32_t brow = (int32_t)((int64_t)g * p.N + n0 + rank * 128);
+        // Gathered A: the A rows of this lane's 4 output rows.  Rows past
+        // the group, padding rows (-1) and invalid indices read row 0; their
+        // promotion multiplies by a zero scale.
+        int32_t ar[4] = {0, 0, 0, 0};
+        if (p.row_map) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int64_t m = m0 + 4 * lane + i;
+                const int32_t r = (m < tr.m_end && m < p.M) ? __ldg(p.row_map + m) : -1;
+                ar[i] = (r >= 0 && r < p.a_rows) ? r : 0;
+            }
+        }
         for (int64_t kb = sg.kb0; kb < sg.kb1; ++kb) {
             if (p.withhold && rank == 1 && it == 1) {   // self-test only
                 ok = false;
@@ -228,7 +247,8 @@ __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, con
             }
             const int s = (int)(it % NS);
             const uint32_t ph = (uint32_t)((it / NS) & 1);
-            if (!mbar_wait(&sh.empty[s], ph ^ 1u, abort, p.timeout_ns)) {
+            // every lane sees the stage free (or the warp gives up together)
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sh.empty[s], ph ^ 1u, abort, p.timeout_ns))) {
                 ok = false;
                 break;
             }
@@ -238,19 +258,28 @@ __device__ void run_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, con
             // Both CTAs' loads complete on the even CTA's barrier, which
             // expects the pair's bytes; the odd CTA only issues its loads.
             const uint32_t bar = mapa_shared(smem_u32(&sh.full[s]), 0);
-            if (rank == 0) mbar_arrive_expect_tx(&sh.full[s], 2 * (A_BYTES + B_BYTES));
-            tma_load_2d_pair(a_dst, tmA, bar, (int32_t)(kb * BK), (int32_t)m0);
-            if (p.b_major == FP8_B_KMAJOR)
-                tma_load_2d_pair(b_dst, tmB, bar, (int32_t)(kb * BK), brow);
-            else
-                tma_load_2d_pair(b_dst, tmB, bar, (int32_t)(n0 + rank * 128), (int32_t)(kb * BK));
+            if (lane == 0 && rank == 0) mbar_arrive_expect_tx(&sh.full[s], 2 * (A_BYTES + B_BYTES));
+            __syncwarp();
+            if (p.row_map) {
+                // 32 gathers of 4 rows each fill the same swizzled 128-row tile
+                tma_gather4_pair(a_dst + lane * 4 * BK, tmA, bar, (int32_t)(kb * BK), ar[0], ar[1],
+                                 ar[2], ar[3]);
+            } else if (lane == 0) {
+                tma_load_2d_pair(a_dst, tmA, bar, (int32_t)(kb * BK), (int32_t)m0);
+            }
+            if (lane == 0) {
+                if (p.b_major == FP8_B_KMAJOR)
+                    tma_load_2d_pair(b_dst, tmB, bar, (int32_t)(kb * BK), brow);
+                else
+                    tma_load_2d_pair(b_dst, tmB, bar, (int32_t)(n0 + rank * 128), (int32_t)(kb * BK));
+            }
         }
     }
     // Every copy issued must land before the CTA may exit: stage s received
     // ceil((it - s) / NS) loads, the last one completing phase (count-1)&1.
     // A pair's loads all count on the even CTA's barriers, so it drains for
     // both (the odd CTA stays resident until the closing cluster barrier).
-    if (rank != 0) return;
+    if (rank != 0 || lane != 0) return;
 #pragma unroll
     for (int s = 0; s < NS; ++s) {
         const int64_t count = it > s ? (it - s + NS - 1) / NS : 0;
@@ -345,8 +374,19 @@ __device__ void run_promotion(const CUtensorMap* tmD, const GemmParams& p, Share
         //   sb   its 128-column block's weight scale (sb_gran 128), or
         //   sb4  4 of its half's 128 column scales (sb_gran 1), staged in this
         //        warp's shared buffer so every lane can read all 128.
-        const float* sa_ptr = p.sA + (row_ok ? m + (int64_t)kb0 * p.M : 0);
-        const int64_t sa_step = row_ok ? p.M : 0;
+        // the row's activation scales: sA[kb][m], or with gathered A the
+        // scales of its A row (none for padding rows: scale 0, output 0)
+        int64_t sa_row = m, sa_ld = p.M;
+        bool sa_ok = row_ok;
+        if (p.row_map) {
+            const int32_t r = row_ok ? __ldg(p.row_map + m) : -1;
+            if (r < -1 || r >= p.a_rows) report_error(FP8_ERR_SHAPE);
+            sa_ok = r >= 0 && r < p.a_rows;
+            sa_row = r;
+            sa_ld = p.a_rows;
+        }
+        const float* sa_ptr = p.sA + (sa_ok ? sa_row + (int64_t)kb0 * sa_ld : 0);
+        const int64_t sa_step = sa_ok ? sa_ld : 0;
         const bool use_sb = active && GRAN == 128;
         const float* sb_ptr = p.sB;
         int64_t sb_step = 0;
@@ -368,7 +408,7 @@ __device__ void run_promotion(const CUtensorMap* tmD, const GemmParams& p, Share
 #pragma unroll
         for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
 
-        float sa_next = row_ok ? __ldg(sa_ptr) : 0.0f;
+        float sa_next = sa_ok ? __ldg(sa_ptr) : 0.0f;
         float sb_next = use_sb ? __ldg(sb_ptr) : 0.0f;
         if (GRAN == 1) {
             *reinterpret_cast<float4*>(&sh.sbw[ew][kb0 & 1][lane * 4]) =
@@ -383,7 +423,7 @@ __device__ void run_promotion(const CUtensorMap* tmD, const GemmParams& p, Share
                 sa_ptr += sa_step;
                 sb_ptr += sb_step;
                 sb4_ptr += sb4_step;
-                if (row_ok) sa_next = __ldg(sa_ptr);
+                if (sa_ok) sa_next = __ldg(sa_ptr);
                 if (use_sb) sb_next = __ldg(sb_ptr);
                 if (use_sb4) sb4_next = __ldg(sb4_ptr);
             }
@@ -588,7 +628,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         regs_dec<CTRL_REGS>();
         if (!sh.bad) {
             if (warp == 0) {
-                if (lane == 0) run_producer(&tmA, &tmB, p, smem, sh, nmb, nnb, nkb);
+                run_producer(&tmA, &tmB, p, smem, sh, nmb, nnb, nkb, lane);
                 __syncwarp();
             } else if (warp == 1 && rank == 0) {   // a pair's MMAs issue from the even CTA
                 if (lane == 0) run_mma(p, smem, sh, nmb, nnb, nkb);
@@ -759,16 +799,22 @@ __global__ void __launch_bounds__(256) k_zero_split_tiles(float* __restrict__ D,
     }
 }
 
+// row_map != nullptr: gathered A (grouped GEMMs), A [a_rows][K] read row by
+// row through row_map[M]; sA [K/128][a_rows].
 int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, int b_major, const float* sB,
                 int sb_gran, int64_t M, int64_t N, int64_t K, const int32_t* group_offsets, int G,
-                void* D, int out_dtype, int64_t ldd, int withhold, cudaStream_t st)
+                void* D, int out_dtype, int64_t ldd, int withhold, const int32_t* row_map,
+                int64_t a_rows, cudaStream_t st)
 {
     if (M == 0) return FP8_OK;
     const GemmDeviceSetup setup = gemm_device_setup();
     if (!setup.ok) return FP8_ERR_LAUNCH;
     if (setup.pair_clusters < 1) return FP8_ERR_DEVICE;   // needs co-scheduled 2-CTA clusters
     CUtensorMap tmA, tmB;
-    if (!make_map(&tmA, A, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, BM)) return FP8_ERR_LAUNCH;
+    // gathered A: boxes one row high, four rows per gather
+    if (!(row_map ? make_map(&tmA, A, (uint64_t)K, (uint64_t)a_rows, (uint64_t)K, BK, 1)
+                  : make_map(&tmA, A, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, BM)))
+        return FP8_ERR_LAUNCH;
     bool okB;
     if (b_major == FP8_B_KMAJOR) {
         const uint64_t rows = (uint64_t)N * (uint64_t)(group_offsets ? G : 1);
@@ -799,6 +845,8 @@ int launch_gemm(const uint8_t* A, const float* sA, const uint8_t* B, int b_major
     p.sb_gran = sb_gran;
     p.out_dtype = out_dtype;
     p.withhold = withhold;
+    p.row_map = row_map;
+    p.a_rows = row_map ? a_rows : M;
     p.band = group_offsets ? BAND_GROUPED : BAND_DENSE;
     p.timeout_ns = wait_timeout_ns();
     // grouped: each group adds at most one partly idle 256-row block
@@ -833,7 +881,16 @@ int launch_blockscaled_gemm(const uint8_t* A, const float* sA, const uint8_t* B,
                             int64_t ldd, cudaStream_t st)
 {
     return launch_gemm(A, sA, B, b_major, sB, sb_gran, M, N, K, group_offsets, G, D, out_dtype,
-                       ldd, 0, st);
+                       ldd, 0, nullptr, 0, st);
+}
+
+int launch_grouped_gemm_gather(const uint8_t* A, const float* sA, int64_t a_rows,
+                               const int32_t* row_map, const uint8_t* B, const float* sB,
+                               const int32_t* group_offsets, int G, int64_t M, int64_t N, int64_t K,
+                               void* D, int out_dtype, cudaStream_t st)
+{
+    return launch_gemm(A, sA, B, FP8_B_KMAJOR, sB, 128, M, N, K, group_offsets, G, D, out_dtype, N,
+                       0, row_map, a_rows, st);
 }
 
 int launch_blockscaled_gemm_withheld(const uint8_t* A, const float* sA, const uint8_t* B,
@@ -842,7 +899,7 @@ int launch_blockscaled_gemm_withheld(const uint8_t* A, const float* sA, const ui
                                      void* D, int out_dtype, int64_t ldd, cudaStream_t st)
 {
     return launch_gemm(A, sA, B, b_major, sB, sb_gran, M, N, K, group_offsets, G, D, out_dtype,
-                       ldd, 1, st);
+                       ldd, 1, nullptr, 0, st);
 }
 
 cudaError_t launch_selftest_wait(cudaStream_t st)

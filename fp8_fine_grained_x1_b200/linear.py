@@ -16,7 +16,8 @@ from it and joined back before the GEMM:
                form and requantized into 128x1 groups
   MoeStep      tokens X[T,K] --1x128, written straight to their expert-
                contiguous, 128-padded FP8 rows-->; W[G,N,K] --128x128-->;
-               grouped GEMM
+               grouped GEMM (or, gather=True, quantized once and gathered by
+               the GEMM)
 
 ("5 Ways You can get More Deepseek While Spending Less", Figure 6: Fprop,
 Dgrad and Wgrad all run in FP8; why-be.co.kr / cameseeing.com posts and
@@ -35,9 +36,10 @@ from __future__ import annotations
 import torch
 
 from . import (B_KMAJOR, B_MNMAJOR, SCALE_FP32, SCALE_POW2, fp8_blockscaled_gemm,
-               fp8_blockscaled_gemm_pow2, fp8_grouped_gemm, fp8_grouped_gemm_pow2,
+               fp8_blockscaled_gemm_pow2, fp8_grouped_gemm, fp8_grouped_gemm_gather,
+               fp8_grouped_gemm_pow2,
                fp8_moe_combine, fp8_moe_dispatch_workspace_bytes, fp8_moe_quant_dispatch,
-               fp8_quant_act_128x1, fp8_quant_act_1x128, fp8_quant_w_128x128,
+               fp8_moe_route, fp8_quant_act_128x1, fp8_quant_act_1x128, fp8_quant_w_128x128,
                fp8_requant_1x128_to_128x1, moe_capacity)
 
 
@@ -215,28 +217,42 @@ class WgradCachedStep:
 
 
 class MoeStep:
-    """MoE expert layer forward: tokens X[T,K] --1x128 quantized straight
-    into expert-contiguous, 128-padded FP8 groups (fp8_moe_quant_dispatch)-->,
-    W[G,N,K] --128x128-->, grouped GEMM.  `combine(weights)` adds the
-    weighted return to token order."""
-    # routing (count, scan, rank), fused quantizer, padding rows, quantize W
-    # (on a side stream), grouped GEMM (+1 memset)
-    kernel_calls = 7
+    """MoE expert layer forward.  Tokens X[T,K] are quantized 1x128 straight
+    into their expert-contiguous, 128-padded rows (fp8_moe_quant_dispatch),
+    W[G,N,K] is quantized 128x128, and the grouped GEMM reads A in place.
+    With gather=True the tokens are instead quantized once in token order,
+    routed without moving rows (fp8_moe_route), and the grouped GEMM reads
+    each row's token codes through TMA gathers (fp8_grouped_gemm_gather): the
+    dispatched copy (k rows per token) is never written, at the price of a
+    slower GEMM (the gathers issue 32 TMA operations per K-block where a
+    tiled load issues one).  `combine(weights)` adds the weighted return to
+    token order."""
 
     def __init__(self, x, topk, w, out_dtype=torch.bfloat16, scale_mode=SCALE_FP32,
-                 tensor_core_scaling=False):
+                 tensor_core_scaling=False, gather=False):
         T, K = x.shape
         G, N, K2 = w.shape
         assert K == K2
         if tensor_core_scaling and scale_mode != SCALE_POW2:
             raise ValueError("tensor-core scaling needs power-of-two scales (SCALE_POW2)")
+        if tensor_core_scaling and gather:
+            raise ValueError("the tensor-core-scaled grouped GEMM reads dispatched rows only")
+        self.gather = gather
         self._gemm = fp8_grouped_gemm_pow2 if tensor_core_scaling else fp8_grouped_gemm
+        # gather: routing (count, scan, rank), token quantizer, weight quantizer
+        # (side stream), gathered grouped GEMM; else routing, fused quantizer,
+        # padding rows, weight quantizer, grouped GEMM (+1 memset either way)
+        self.kernel_calls = 6 if self.gather else 7
         k = topk.shape[1]
         d = x.device
         self.x, self.topk, self.w, self.mode, self.G = x, topk, w, scale_mode, G
         self.M_cap = moe_capacity(T, k, G)
-        self.qa = _empty((self.M_cap, K), torch.uint8, d)
-        self.sa = _empty((K // 128, self.M_cap), torch.float32, d)
+        if self.gather:
+            self.qx = _empty((T, K), torch.uint8, d)
+            self.sx = _empty((K // 128, T), torch.float32, d)
+        else:
+            self.qa = _empty((self.M_cap, K), torch.uint8, d)
+            self.sa = _empty((K // 128, self.M_cap), torch.float32, d)
         self.offsets = _empty((G + 1,), torch.int32, d)
         self.token_row = _empty((T, k), torch.int32, d)
         self.row_token = _empty((self.M_cap,), torch.int32, d)
@@ -247,7 +263,7 @@ class MoeStep:
         self.out = None
         self.inputs, self.output = [x, w, topk], self.y
         # the weight quantizer on the side stream: the short routing kernels
-        # of the token path overlap it
+        # and the token path overlap it
         self._fork = _Fork(d)
 
     def quantize(self, stream=None):
@@ -255,12 +271,21 @@ class MoeStep:
         G, N, K = self.w.shape
         fp8_quant_w_128x128(self.w.view(G * N, K), self.qw.view(G * N, K),
                             self.sw.view(G * N // 128, K // 128), self.mode, side)
-        fp8_moe_quant_dispatch(self.x, self.topk, self.G, self.qa, self.sa, self.offsets,
-                               self.token_row, self.row_token, self.ws, self.mode, cur)
+        if self.gather:
+            fp8_moe_route(self.topk, self.G, self.offsets, self.token_row, self.row_token, self.ws,
+                          cur)
+            fp8_quant_act_1x128(self.x, self.qx, self.sx, self.mode, cur)
+        else:
+            fp8_moe_quant_dispatch(self.x, self.topk, self.G, self.qa, self.sa, self.offsets,
+                                   self.token_row, self.row_token, self.ws, self.mode, cur)
         self._fork.end(cur)
 
     def gemm(self, stream=None):
-        self._gemm(self.qa, self.sa, self.qw, self.sw, self.offsets, self.y, stream)
+        if self.gather:
+            fp8_grouped_gemm_gather(self.qx, self.sx, self.row_token, self.qw, self.sw,
+                                    self.offsets, self.y, stream)
+        else:
+            self._gemm(self.qa, self.sa, self.qw, self.sw, self.offsets, self.y, stream)
 
     def combine(self, weights, stream=None):
         T = self.x.shape[0]

@@ -225,6 +225,32 @@ int fp8_grouped_gemm(const uint8_t* A, const float* sA, const uint8_t* B, const 
                      void* D, int out_dtype, void* stream);
 
 /*
+ * fp8_grouped_gemm with A gathered from per-token rows instead of read from
+ * an expert-ordered copy ([P1]/[P3] MoE activations move in FP8; [P5] each
+ * group loads one expert's weights): output row m of D is the product of A
+ * row row_token[m] with its expert's weight, so the dispatched rows are never
+ * written to memory.  The tensor cores read the rows through TMA gathers.
+ * It saves the k-fold copy of the token rows in HBM (and the traffic of
+ * writing it) but not time: a K-block's 128 rows take 32 four-row gathers
+ * where a tiled load takes one TMA operation, and on the MoE workload (16384
+ * tokens, top-8, 32 experts, N = 2048, K = 7168) this GEMM ran 2.3x as long
+ * as fp8_grouped_gemm on the dispatched rows.
+ *   A        [T][K] E4M3 codes of the tokens (1x128 groups), row-major
+ *   sA       [K/128][T] FP32, their scales
+ *   row_token [M_total] int32 in DEVICE memory: the A row of each output row,
+ *            -1 for padding rows, whose output is 0 (fp8_moe_route's
+ *            row_token has this layout).  An entry below -1 or at or beyond T
+ *            is treated as padding and records FP8_ERR_SHAPE.
+ *   B, sB, group_offsets, G, M_total, N, K, D, out_dtype as fp8_grouped_gemm.
+ * Sizes: as fp8_grouped_gemm, plus 1 <= T <= 2^31 - 1 when M_total > 0.
+ * row_token 4-byte aligned.  One kernel launch.
+ */
+int fp8_grouped_gemm_gather(const uint8_t* A, const float* sA, int64_t T, const int32_t* row_token,
+                            const uint8_t* B, const float* sB, const int32_t* group_offsets, int G,
+                            int64_t M_total, int64_t N, int64_t K, void* D, int out_dtype,
+                            void* stream);
+
+/*
  * FP8 dispatch of MoE activations ([P1]/[P3] cache and dispatch activations
  * in FP8; [P4] top-8 routing): rows of 1x128-quantized tokens, with their
  * scales, are gathered into expert-contiguous groups, each padded with zero
@@ -256,6 +282,17 @@ int fp8_moe_dispatch(const uint8_t* q, const float* sA, int64_t T, int64_t K, co
                      int k, int G, uint8_t* q_out, float* sA_out, int64_t M_cap,
                      int32_t* group_offsets, int32_t* token_row, int32_t* row_token,
                      void* workspace, int64_t workspace_bytes, void* stream);
+
+/*
+ * The routing half of fp8_moe_dispatch alone: group_offsets, token_row and
+ * row_token exactly as fp8_moe_dispatch writes them, and no rows moved (for
+ * fp8_grouped_gemm_gather, which reads the token rows through row_token).
+ * Arguments, sizes, workspace and errors as fp8_moe_dispatch without q, sA,
+ * K, q_out and sA_out.  Launches three kernels and one memset.
+ */
+int fp8_moe_route(const int32_t* topk, int64_t T, int k, int G, int64_t M_cap,
+                  int32_t* group_offsets, int32_t* token_row, int32_t* row_token, void* workspace,
+                  int64_t workspace_bytes, void* stream);
 
 /*
  * 1x128 quantization of the tokens fused with their FP8 dispatch ([P5]

@@ -180,10 +180,17 @@ def test_moe_grouped_fprop(pow2_tc):
     qw = qw.reshape(G, N, K)
     sw = sw.reshape(G, N // 128, K // 128)
 
-    # dispatched rows: the oracle's dispatch of the oracle's codes, bit-exact
+    # the oracle's dispatch of the oracle's codes: the rows the GEMM must see;
+    # the step holds them dispatched (tensor-core scaling) or reads them
+    # through row_token from the tokens' own codes (gather), bit-exact either way
     od = omoe.moe_dispatch(qx, sx, topk.numpy(), G, step.M_cap)
-    assert np.array_equal(step.qa.cpu().numpy(), od["q"])
-    assert np.array_equal(step.sa.cpu().numpy(), od["sA"])
+    if step.gather:
+        assert np.array_equal(step.qx.cpu().numpy(), qx)
+        assert np.array_equal(step.sx.cpu().numpy(), sx)
+        assert np.array_equal(step.row_token.cpu().numpy(), od["row_token"])
+    else:
+        assert np.array_equal(step.qa.cpu().numpy(), od["q"])
+        assert np.array_equal(step.sa.cpu().numpy(), od["sA"])
 
     # GEMM at the first, last-real and last-padding row of every expert + random rows
     rng = np.random.default_rng(4)
