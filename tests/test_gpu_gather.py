@@ -154,3 +154,24 @@ def test_gather_rejects_bad_arguments():
                                        128, P(D), 1, None) == fg.FP8_OK
     assert fg.fp8_get_status() == fg.FP8_OK
     assert torch.all(D == 0).item()
+
+
+def test_moe_step_with_gather_equals_the_default_step():
+    """MoeStep(gather=True) (route, quantize tokens once, gathered GEMM) and
+    the default step (fused quantize-and-dispatch, grouped GEMM) give the
+    same output bit for bit, and the same routing."""
+    from fp8_fine_grained_x1_b200 import linear
+    T, k, G, N, K = 1024, 8, 16, 256, 512
+    x = synth.activations(T, K, seed=31, outlier_seed=32).to(dev())
+    topk = to_dev(synth.zipf_topk_routing(T, G, k, seed=33).numpy().astype(np.int32))
+    w = synth.normal((G, N, K), 0.006, 34).to(dev())
+    a = linear.MoeStep(x, topk, w)
+    b = linear.MoeStep(x, topk, w, gather=True)
+    ya, yb = a(), b()
+    torch.cuda.synchronize()
+    assert fg.fp8_get_status() == fg.FP8_OK
+    assert b.kernel_calls == 6 and a.kernel_calls == 7
+    assert torch.equal(a.offsets, b.offsets) and torch.equal(a.row_token, b.row_token)
+    assert torch.equal(a.token_row, b.token_row)
+    used = int(a.offsets[-1].item())                              # rows past off[G] are not written
+    assert torch.equal(ya[:used].view(torch.int16), yb[:used].view(torch.int16))
