@@ -104,15 +104,15 @@ def gemm_roofline(gemm_tflops: float, clocks: dict, peaks: dict) -> dict:
 
 
 def targets(roof: dict, quant_gbs: float) -> dict:
-    """The two targets of the path and the fraction each is judged on: the
+    """The two targets of the path and the fraction each is measured against: the
     GEMM against the dense FP8 spec (4.5 PFLOP/s, >= 60 %), the quantizers
     against the HBM spec (8 TB/s, >= 75 %).  The measured-peak fractions in
     `roofline` and `quantizers` are the engineering view beside them."""
     g = roof["achieved"] / FP8_SPEC_TFLOPS
     q = quant_gbs / HBM_SPEC_GBS
-    return {"gemm": {"judged_on": f"achieved / {FP8_SPEC_TFLOPS} TFLOP/s dense FP8 spec",
+    return {"gemm": {"measured_against": f"achieved / {FP8_SPEC_TFLOPS} TFLOP/s dense FP8 spec",
                      "frac": g, "threshold": 0.60, "met": g >= 0.60},
-            "quantizers": {"judged_on": f"achieved / {HBM_SPEC_GBS} GB/s HBM spec",
+            "quantizers": {"measured_against": f"achieved / {HBM_SPEC_GBS} GB/s HBM spec",
                            "frac": q, "threshold": 0.75, "met": q >= 0.75}}
 
 

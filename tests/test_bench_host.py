@@ -44,7 +44,7 @@ def test_both_arms_print_the_same_config():
     assert desc == {"workload": "w", "M": 1, "N": 2, "K": 3}
 
 
-def test_targets_name_the_spec_fractions_they_are_judged_on():
+def test_targets_name_the_spec_fractions_they_are_measured_against():
     roof = bench.gemm_roofline(2800.0, {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}, PEAKS)
     t = bench.targets(roof, 6100.0)
     assert abs(t["gemm"]["frac"] - 2800.0 / 4500.0) < 1e-12 and t["gemm"]["met"]
@@ -52,4 +52,4 @@ def test_targets_name_the_spec_fractions_they_are_judged_on():
     t = bench.targets(bench.gemm_roofline(1900.0, {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0,
                                                     "reasons": []}, PEAKS), 4500.0)
     assert not t["gemm"]["met"] and not t["quantizers"]["met"]
-    assert "4500" in t["gemm"]["judged_on"] and "8000" in t["quantizers"]["judged_on"]
+    assert "4500" in t["gemm"]["measured_against"] and "8000" in t["quantizers"]["measured_against"]
